@@ -1,0 +1,72 @@
+"""ctypes view of libfa_b200.so (the C ABI declared in include/fa.h).
+
+Loading fails loudly if the library has not been built; there is no
+fallback implementation anywhere in the package.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libfa_b200.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_CUDA = 3
+FA_ERR_DEVICE_TIMEOUT = 4
+FA_BF16 = 0
+FA_F32 = 1
+
+c_void_p = ctypes.c_void_p
+c_int = ctypes.c_int
+c_ll = ctypes.c_longlong
+c_float = ctypes.c_float
+c_size_t = ctypes.c_size_t
+
+# name -> (restype, argtypes), one entry per function in include/fa.h
+SIGNATURES = {
+    "fa_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                       c_int, c_int, c_int, c_int, c_float, c_void_p, c_int, c_ll, c_void_p]),
+    "fa_bwd_workspace_size": (c_size_t, [c_ll, c_int, c_int, c_int]),
+    "fa_bwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                       c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                       c_float, c_void_p, c_int, c_ll, c_void_p, c_size_t, c_void_p]),
+    "fa_get_error_string": (ctypes.c_char_p, [c_int]),
+    "fa_check_device_error": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_uint)]),
+    "fa_set_wait_budget": (None, [c_ll]),
+    "fa_selftest_wait_timeout": (c_int, [c_ll, c_void_p]),
+    "fa_version": (c_int, []),
+}
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = lib().fa_get_error_string(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{what}: {msg}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded once)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_tmem_b200.build`"
+                " (the package has no non-CUDA fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def check(status: int, what: str) -> None:
+    if status != FA_OK:
+        raise FAError(status, what)

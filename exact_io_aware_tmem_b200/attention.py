@@ -1,0 +1,126 @@
+"""Python entry points over the C ABI (argument marshalling only).
+
+Every step of the forward and backward passes runs in the CUDA kernels of
+libfa_b200.so; this module checks torch tensors, allocates the outputs with
+torch (device memory and streams are all PyTorch provides), and passes raw
+pointers and the current stream to ``fa_fwd`` / ``fa_bwd``.
+
+Layouts (token-major, as in include/fa.h):
+  dense : q [B, N, H, D], k / v [B, N, H_kv, D]; lse [B, H, N]
+  packed: q [T, H, D],    k / v [T, H_kv, D] with cu_seqlens int32 [B+1]
+          on the device; lse [H, T]
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import _abi
+
+_DTYPES = {torch.bfloat16: _abi.FA_BF16, torch.float32: _abi.FA_F32}
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _shape(q: torch.Tensor, k: torch.Tensor, cu_seqlens, max_seqlen):
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {q.dtype}; use bfloat16 or float32")
+    for t in (q, k):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if cu_seqlens is None:
+        if q.dim() != 4 or k.dim() != 4:
+            raise ValueError("dense inputs are [B, N, H, D]")
+        B, N, H, D = q.shape
+        H_kv = k.shape[2]
+        return B, N, H, H_kv, D, 0, B * N
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("packed inputs are [T, H, D]")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+        raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+    T, H, D = q.shape
+    if max_seqlen is None:
+        raise ValueError("packed inputs need max_seqlen")
+    return cu_seqlens.numel() - 1, 0, H, k.shape[1], D, int(max_seqlen), T
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = False,
+        scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+        max_seqlen: Optional[int] = None, out: Optional[torch.Tensor] = None,
+        lse: Optional[torch.Tensor] = None):
+    """Attention forward. Returns (O, LSE)."""
+    B, N, H, H_kv, D, max_sl, T = _shape(q, k, cu_seqlens, max_seqlen)
+    if v.shape != k.shape or v.dtype != q.dtype or k.dtype != q.dtype:
+        raise ValueError("k and v must match in shape and dtype with q's dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N) if cu_seqlens is None else (H, T), device=q.device,
+                          dtype=torch.float32)
+    s = -1.0 if scale is None else float(scale)
+    st = _abi.lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, N, D,
+                           _DTYPES[q.dtype], int(bool(causal)), s, _ptr(cu_seqlens), max_sl, T,
+                           _stream(q.device))
+    _abi.check(st, "fa_fwd")
+    return out, lse
+
+
+def workspace_size(T: int, H: int, D: int, dtype: torch.dtype) -> int:
+    return int(_abi.lib().fa_bwd_workspace_size(T, H, D, _DTYPES[dtype]))
+
+
+def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+        o: torch.Tensor, lse: torch.Tensor, *, causal: bool = False,
+        scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+        max_seqlen: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+        dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+        dv: Optional[torch.Tensor] = None):
+    """Attention backward for the loss sum(O * dO). Returns (dQ, dK, dV)."""
+    B, N, H, H_kv, D, max_sl, T = _shape(q, k, cu_seqlens, max_seqlen)
+    for t in (dout, o, v, lse):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = workspace_size(T, H, D, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    s = -1.0 if scale is None else float(scale)
+    st = _abi.lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                           _ptr(dk), _ptr(dv), B, H, H_kv, N, D, _DTYPES[q.dtype],
+                           int(bool(causal)), s, _ptr(cu_seqlens), max_sl, T, _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(q.device))
+    _abi.check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def check_device_error(device: Optional[torch.device] = None) -> tuple:
+    """Synchronise the current stream; return (status, where) and clear the flag."""
+    import ctypes
+    dev = torch.device("cuda") if device is None else device
+    where = ctypes.c_uint(0)
+    st = _abi.lib().fa_check_device_error(_stream(dev), ctypes.byref(where))
+    return st, where.value
+
+
+def selftest_wait_timeout(cycles: int, device: Optional[torch.device] = None) -> None:
+    dev = torch.device("cuda") if device is None else device
+    _abi.check(_abi.lib().fa_selftest_wait_timeout(int(cycles), _stream(dev)),
+               "fa_selftest_wait_timeout")
+
+
+def set_wait_budget(cycles: int) -> None:
+    _abi.lib().fa_set_wait_budget(int(cycles))
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

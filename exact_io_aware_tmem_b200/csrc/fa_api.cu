@@ -1,0 +1,255 @@
+// C ABI of libfa_b200.so (declared in include/fa.h): host-side argument
+// checks, dispatch to the kernels, tensor-map encoding and the device error
+// word that bounded in-kernel waits report through.
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "params.h"
+
+namespace fa {
+
+// Word 0: error bits (ERR_TIMEOUT, ERR_BOUNDS); word 1: code of the wait or
+// check that failed. Every kernel receives its address in AttnParams::err.
+__device__ unsigned g_err_word[2];
+
+namespace {
+
+constexpr long long kDefaultBudget = 4000000000LL;  // ~2 s at 1.9 GHz
+long long g_budget = kDefaultBudget;
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+
+// Device address of g_err_word on the current device (looked up once).
+unsigned* err_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_err_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<unsigned*>(ptr);
+  }
+  return g_err_ptr[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Shared checks of fa_fwd / fa_bwd; fills the size fields of ``p``.
+fa_status check_common(AttnParams& p, int B, int H, int H_kv, int N, int D, fa_dtype dtype,
+                       int causal, float scale, const int* cu_seqlens, int max_seqlen,
+                       long long total_tokens) {
+  if (B < 0 || H <= 0 || H_kv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (H % H_kv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  if (dtype == FA_BF16 && D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_F32 && D > 128) return FA_ERR_UNSUPPORTED;
+  if (H > 65535 || B > 65535) return FA_ERR_UNSUPPORTED;  // grid y / z limits
+  if (cu_seqlens != nullptr) {
+    if (max_seqlen < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return FA_ERR_INVALID_ARG;
+    if (B == 0 && total_tokens != 0) return FA_ERR_INVALID_ARG;
+    p.max_seqlen = max_seqlen;
+    p.total = total_tokens;
+    p.N = 0;
+  } else {
+    if (N < 0) return FA_ERR_INVALID_ARG;
+    const long long total = static_cast<long long>(B) * N;
+    if (total > INT32_MAX) return FA_ERR_UNSUPPORTED;
+    p.max_seqlen = N;
+    p.total = total;
+    p.N = N;
+  }
+  p.cu_seqlens = cu_seqlens;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.D = D;
+  p.causal = causal;
+  if (!(scale > 0.f) || !isfinite(scale)) scale = 1.f / sqrtf(static_cast<float>(D));
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err.word = nullptr;
+  p.err.budget = g_budget;
+  return FA_OK;
+}
+
+}  // namespace
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long rows,
+                       unsigned long long cols, unsigned box_cols, unsigned box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};  // bytes between rows
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
+__global__ void wait_selftest_kernel(DevErr e) {
+  __shared__ alignas(8) unsigned long long bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on ``bar``: the wait must give up on its own.
+  mbar_wait(smem_u32(&bar), 0, e, &abort_flag, 0x5e1f7e57u);
+}
+
+}  // namespace
+
+cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(err);
+  return cudaGetLastError();
+}
+
+}  // namespace fa
+
+using fa::AttnParams;
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int H_kv, int N, int D, fa_dtype dtype, int causal, float scale,
+                 const int* cu_seqlens, int max_seqlen, long long total_tokens,
+                 fa_stream_t stream) {
+  AttnParams p = {};
+  fa_status st = fa::check_common(p, B, H, H_kv, N, D, dtype, causal, scale, cu_seqlens,
+                                  max_seqlen, total_tokens);
+  if (st != FA_OK) return st;
+  if (p.total == 0 || p.max_seqlen == 0 || B == 0) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!fa::aligned16(q) || !fa::aligned16(k) || !fa::aligned16(v) || !fa::aligned16(o))
+    return FA_ERR_INVALID_ARG;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.lse = lse;
+  p.err.word = fa::err_word();
+  if (p.err.word == nullptr) return FA_ERR_CUDA;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = (dtype == FA_F32) ? fa::launch_fwd_f32(p, s) : fa::launch_fwd_bf16(p, s);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype) {
+  if (total_tokens < 0 || H <= 0 || D <= 0) return 0;
+  const size_t T = static_cast<size_t>(total_tokens);
+  const size_t dq = (dtype == FA_BF16) ? fa::round256(T * H * D * sizeof(float)) : 0;
+  return dq + fa::round256(T * H * sizeof(float)) + 256;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+                 int D, fa_dtype dtype, int causal, float scale, const int* cu_seqlens,
+                 int max_seqlen, long long total_tokens, void* workspace, size_t ws_bytes,
+                 fa_stream_t stream) {
+  AttnParams p = {};
+  fa_status st = fa::check_common(p, B, H, H_kv, N, D, dtype, causal, scale, cu_seqlens,
+                                  max_seqlen, total_tokens);
+  if (st != FA_OK) return st;
+  if (p.total == 0 || p.max_seqlen == 0 || B == 0) return FA_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!fa::aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  if (ws_bytes < fa_bwd_workspace_size(p.total, H, D, dtype)) return FA_ERR_INVALID_ARG;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = const_cast<void*>(o);
+  p.lse = const_cast<float*>(lse);
+  p.dout = dout;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t T = static_cast<size_t>(p.total);
+  if (dtype == FA_BF16) {
+    p.dq_accum = reinterpret_cast<float*>(ws);
+    ws += fa::round256(T * H * D * sizeof(float));
+  }
+  p.delta = reinterpret_cast<float*>(ws);
+  p.err.word = fa::err_word();
+  if (p.err.word == nullptr) return FA_ERR_CUDA;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = (dtype == FA_F32) ? fa::launch_bwd_f32(p, s) : fa::launch_bwd_bf16(p, s);
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+const char* fa_get_error_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: bad pointer, size, alignment or layout";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: no kernel for this dtype / head dim / size";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a bounded in-kernel wait ran out";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_check_device_error(fa_stream_t stream, unsigned* where) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  unsigned w[2] = {0, 0};
+  if (cudaMemcpyFromSymbol(w, fa::g_err_word, sizeof(w)) != cudaSuccess) return FA_ERR_CUDA;
+  if (where != nullptr) *where = w[1];
+  if (w[0] == 0) return FA_OK;
+  const unsigned zero[2] = {0, 0};
+  if (cudaMemcpyToSymbol(fa::g_err_word, zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+  if (w[0] & fa::ERR_TIMEOUT) return FA_ERR_DEVICE_TIMEOUT;
+  return FA_ERR_INVALID_ARG;  // ERR_BOUNDS: cu_seqlens inconsistent with the sizes
+}
+
+void fa_set_wait_budget(long long cycles) {
+  fa::g_budget = cycles > 0 ? cycles : fa::kDefaultBudget;
+}
+
+fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream) {
+  fa::DevErr e{fa::err_word(), cycles > 0 ? cycles : 1000000};
+  if (e.word == nullptr) return FA_ERR_CUDA;
+  return fa::launch_wait_selftest(e, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

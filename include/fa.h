@@ -1,0 +1,177 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) exact-attention library libfa_b200.so.
+ *
+ * The library computes exact scaled dot-product attention
+ *     O = softmax(scale * Q K^T) V
+ * tile by tile with the online-softmax recurrence (running row max m, running
+ * exponential sum l, rescaling of the output accumulator, one division by l at
+ * the end), and saves the row log-sum-exp for the backward pass. The backward
+ * pass recomputes S and P from Q, K and the saved log-sum-exp and forms dV, dP,
+ * dS, dQ and dK; no N x N matrix is ever written to global memory.
+ *
+ * Sources for what is computed:
+ *   - aiqz.cc "Flash Attention V2/V3 optimization", section "IO bottleneck
+ *     analysis" (the attention definition) and section "V2 algorithm
+ *     optimisation", update steps 1-5 (m, l and O recurrence, final O / l);
+ *   - airsota.com interview card (p=1562), section 3 (safe, online softmax)
+ *     and section 4 items 1-3 (deferred normalisation, recomputation from the
+ *     saved statistics, grouped-query attention);
+ *   - agentalpha.top "flash attention" answer, section 2 (recomputation in
+ *     the backward pass);
+ *   - "Flash Attention self-test" (book.bogosort.top), sections C and D, which
+ *     ask for causal masks, variable-length batches, the 1/sqrt(d) scale and
+ *     the dV/dP/dS/dQ/dK relations without answering them; the readings used
+ *     are stated at each entry point below.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout (token-major, contiguous, row-major):
+ *   q, o, dout, dq : [T, H, D]      k, v, dk, dv : [T, H_kv, D]
+ *   where T = B * N for a dense batch, or T = total_tokens (= cu_seqlens[B])
+ *   for a packed variable-length batch.
+ *   lse : float32, [B, H, N] for a dense batch, [H, T] for a packed batch.
+ * Element type (dtype): FA_BF16 (bf16 in and out, fp32 accumulation, tensor
+ *   cores; D must be 64 or 128) or FA_F32 (fp32 everywhere, CUDA cores;
+ *   1 <= D <= 128).
+ * Grouped-query attention: H % H_kv == 0; query head h reads key/value head
+ *   h / (H / H_kv). H_kv == 1 is multi-query attention.
+ * Causal mask: key j is visible to query i iff j <= i, with i and j counted
+ *   from the start of their own sequence. The diagonal is kept.
+ * Variable length: cu_seqlens (device int32, B + 1 non-decreasing entries,
+ *   cu_seqlens[0] == 0) gives sequence b the rows [cu[b], cu[b+1]) of every
+ *   tensor; attention never crosses a sequence boundary; empty sequences are
+ *   allowed. max_seqlen must be >= every length; total_tokens == cu[B].
+ *   With cu_seqlens == NULL the batch is dense and N is the length.
+ * scale: multiplies Q K^T before the row max. scale <= 0 (or NaN) selects
+ *   1 / sqrt(D).
+ * LSE: natural-log log-sum-exp of the scaled logits of each query row,
+ *   LSE_i = m_i + ln(l_i).
+ * Pointers: device pointers, 16-byte aligned (tensor-memory-accelerator
+ *   copies need it). Buffers are owned by the caller; the library allocates
+ *   no device memory and keeps no per-call state.
+ * Streams: every entry point only enqueues work on ``stream`` (NULL = the
+ *   legacy default stream) and returns without synchronising, except
+ *   fa_check_device_error.
+ * Errors: argument errors are detected on the host before anything is
+ *   enqueued and return FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED. Launch
+ *   failures return FA_ERR_CUDA. Every wait inside a kernel is bounded; a wait
+ *   that runs out sets a device error word, which fa_check_device_error
+ *   reports as FA_ERR_DEVICE_TIMEOUT. Nothing traps.
+ */
+#ifndef EXACT_IO_AWARE_TMEM_FA_H
+#define EXACT_IO_AWARE_TMEM_FA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,    /* bad pointer, size, alignment or layout       */
+  FA_ERR_UNSUPPORTED = 2,    /* valid request this build has no kernel for  */
+  FA_ERR_CUDA = 3,           /* a CUDA runtime call or kernel launch failed  */
+  FA_ERR_DEVICE_TIMEOUT = 4  /* a bounded in-kernel wait ran out            */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA
+ * include. */
+typedef struct CUstream_st* fa_stream_t;
+
+/*
+ * fa_fwd - attention forward pass.
+ *
+ * Inputs q, k, v; outputs o (same dtype as q) and lse (float32). Implements
+ * the online-softmax forward of aiqz.cc "Flash Attention V2/V3 optimization",
+ * section "V2 algorithm optimisation" (steps 1-5) with the log-sum-exp saved
+ * as the airsota.com card, section 4 item 2, keeps "m, l" for the backward.
+ *
+ *   B            batch size (number of sequences when cu_seqlens != NULL)
+ *   H, H_kv      query heads and key/value heads (H % H_kv == 0)
+ *   N            sequence length of a dense batch (ignored when packed)
+ *   D            head dimension
+ *   causal       0 or 1
+ *   cu_seqlens   NULL (dense) or device int32[B + 1] (packed)
+ *   max_seqlen   packed only: upper bound on every sequence length
+ *   total_tokens packed only: cu_seqlens[B], the row count of every tensor
+ *
+ * Returns FA_OK once the work is enqueued.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int H_kv, int N, int D, fa_dtype dtype, int causal, float scale,
+                 const int* cu_seqlens, int max_seqlen, long long total_tokens,
+                 fa_stream_t stream);
+
+/*
+ * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs for T tokens,
+ * H query heads and head dimension D: the float32 dQ accumulator [T, H, D]
+ * (bf16 only) and the float32 row terms D_i = dO_i . O_i [H, T], each
+ * rounded up to 256 bytes. Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype);
+
+/*
+ * fa_bwd - attention backward pass for the loss sum(O * dO).
+ *
+ * Recomputes S = scale Q K^T and P = exp(S - LSE) tile by tile from q, k and
+ * the lse that fa_fwd wrote (agentalpha.top "flash attention" answer, section
+ * 2; airsota.com card, section 4 item 2), then forms
+ *   dV = P^T dO, dP = dO V^T, D_i = dO_i . O_i, dS = P * (dP - D_i),
+ *   dQ = scale dS K, dK = scale dS^T Q
+ * (the relations the "Flash Attention self-test", section D, asks for). With
+ * grouped-query attention dk and dv of a key/value head are summed over the
+ * query heads that share it.
+ *
+ *   q, k, v, o, lse, dout   inputs, as written / read by fa_fwd
+ *   dq, dk, dv              outputs, same dtype and layout as q, k, v
+ *   workspace, ws_bytes     caller-owned device scratch of at least
+ *                           fa_bwd_workspace_size(T, H, D, dtype) bytes,
+ *                           256-byte aligned; its contents on entry do not
+ *                           matter and are undefined on return
+ * The remaining arguments mean what they mean for fa_fwd and must match the
+ * forward call that produced o and lse.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+                 int D, fa_dtype dtype, int causal, float scale, const int* cu_seqlens,
+                 int max_seqlen, long long total_tokens, void* workspace, size_t ws_bytes,
+                 fa_stream_t stream);
+
+/* fa_get_error_string - static, human-readable name of a status code. */
+const char* fa_get_error_string(fa_status status);
+
+/*
+ * fa_check_device_error - synchronises ``stream``, then reports and clears
+ * the device error word of the current device: FA_ERR_DEVICE_TIMEOUT if a
+ * kernel's bounded wait ran out since the last check, FA_ERR_CUDA if the
+ * synchronisation failed, else FA_OK. ``where`` (nullable) receives the code
+ * of the wait that gave up.
+ */
+fa_status fa_check_device_error(fa_stream_t stream, unsigned* where);
+
+/*
+ * fa_set_wait_budget - how many SM clock cycles one in-kernel wait may spin
+ * before it gives up (default 4e9, about two seconds). Values <= 0 restore
+ * the default. Applies to launches enqueued after the call.
+ */
+void fa_set_wait_budget(long long cycles);
+
+/*
+ * fa_selftest_wait_timeout - enqueues one small kernel that waits on an
+ * mbarrier no thread ever arrives on, with a budget of ``cycles``, so that
+ * the bounded-wait path can be exercised without faulting or hanging the
+ * GPU. After it, fa_check_device_error must return FA_ERR_DEVICE_TIMEOUT.
+ */
+fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream);
+
+/* fa_version - library version as major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_TMEM_FA_H */
