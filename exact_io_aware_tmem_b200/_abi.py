@@ -33,6 +33,10 @@ SIGNATURES = {
     "fa_bwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                        c_float, c_void_p, c_int, c_ll, c_void_p, c_size_t, c_void_p]),
+    "fa_bwd_phases": (c_int, [ctypes.c_uint, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                              c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                              c_int, c_int, c_int, c_float, c_void_p, c_int, c_ll, c_void_p,
+                              c_size_t, c_void_p]),
     "fa_get_error_string": (ctypes.c_char_p, [c_int]),
     "fa_check_device_error": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_uint)]),
     "fa_set_wait_budget": (None, [c_ll]),

@@ -82,8 +82,12 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
         max_seqlen: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
         dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
-        dv: Optional[torch.Tensor] = None):
-    """Attention backward for the loss sum(O * dO). Returns (dQ, dK, dV)."""
+        dv: Optional[torch.Tensor] = None, phases: int = 7):
+    """Attention backward for the loss sum(O * dO). Returns (dQ, dK, dV).
+
+    ``phases`` selects the kernels to enqueue (bit 0 preprocess, bit 1 main,
+    bit 2 dQ conversion); the default runs all three.
+    """
     B, N, H, H_kv, D, max_sl, T = _shape(q, k, cu_seqlens, max_seqlen)
     for t in (dout, o, v, lse):
         if not t.is_cuda or not t.is_contiguous():
@@ -95,10 +99,12 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     s = -1.0 if scale is None else float(scale)
-    st = _abi.lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
-                           _ptr(dk), _ptr(dv), B, H, H_kv, N, D, _DTYPES[q.dtype],
-                           int(bool(causal)), s, _ptr(cu_seqlens), max_sl, T, _ptr(workspace),
-                           workspace.numel() * workspace.element_size(), _stream(q.device))
+    st = _abi.lib().fa_bwd_phases(int(phases), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                  _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, H_kv, N, D,
+                                  _DTYPES[q.dtype], int(bool(causal)), s, _ptr(cu_seqlens),
+                                  max_sl, T, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  _stream(q.device))
     _abi.check(st, "fa_bwd")
     return dq, dk, dv
 

@@ -1,8 +1,547 @@
-// Attention backward, bf16 on the sm_100a tensor cores (not built yet).
+// Attention backward, bf16 in / fp32 accumulate, on the sm_100a tensor cores.
+//
+// What it computes, for the loss sum(O * dO): the backward pass rebuilds the
+// scores and probabilities from Q, K and the saved LSE instead of storing the
+// N x N matrix (agentalpha.top "flash attention" answer, section 2; airsota.com
+// card, section 4 item 2), then applies the gradient relations the "Flash
+// Attention self-test" (book.bogosort.top, section D) asks for:
+//     P = exp(scale Q K^T - LSE),   dV = P^T dO,   dP = dO V^T,
+//     D_i = dO_i . O_i,   dS = P * (dP - D),   dQ = scale dS K,   dK = scale dS^T Q.
+//
+// Three kernels, in stream order:
+//   bwd_preprocess   D_i = dO_i . O_i (fp32, [H, T]) and zeroes the fp32 dQ
+//                    accumulator [T, H, D]; HBM-bound.
+//   bwd_main         one CTA per (sequence, key/value head, 128-key tile j);
+//                    K_j and V_j stay in shared memory while the CTA walks
+//                    every 64-row query tile i of every query head of the
+//                    group (GQA dK/dV accumulate in TMEM, no extra reduction).
+//                    Per step, in TMEM (keys on the 128 lanes):
+//                      S^T  = K_j Q_i^T              (M=128 keys, N=64, K=D)
+//                      P^T  = exp2(S^T c - LSE_i log2 e), masked, bf16 over S^T
+//                      dV  += P^T dO_i               (A = P^T from TMEM)
+//                      dP^T = V_j dO_i^T
+//                      dS^T = P^T * (dP^T - D_i)  -> bf16 in shared memory
+//                      dK  += dS^T Q_i
+//                      dQ_i^T = K_j^T dS^T           (M=128 = D lanes, N=64)
+//                    and the dQ^T tile is added into the fp32 accumulator
+//                    by per-element red.global.add.f32 (the separate
+//                    dQ-accumulation path); dK, dV are scaled and stored at
+//                    the end.
+//   bwd_dq_convert   dQ = bf16(scale * accumulator).
+//
+// Roles in bwd_main (320 threads): warps 0-3 softmax / dS (thread = key row
+// = TMEM lane) and the dK/dV epilogue; warps 4-7 dQ drain (thread = head-dim
+// row of dQ^T); warp 8 TMA producer; warp 9 MMA issuer.
+// TMEM columns: dV [0,128) dK [128,256) S/P [256,320) dP [320,384)
+//               dQ^T x2 [384,512).
+// D = 64 runs the same kernel: the tensor maps are 3-D (D, heads, tokens), so
+// the second 64-wide column block is out of bounds and arrives as zeros.
+#include <limits.h>
+#include <math.h>
+
+#include <algorithm>
+
 #include "params.h"
 
 namespace fa {
+namespace {
 
-cudaError_t launch_bwd_bf16(const AttnParams&, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int BN = 128;  // keys per CTA (TMEM lanes)
+constexpr int BM = 64;   // query rows per step
+constexpr int DP = 128;  // padded head dim
+constexpr int QS = 2;    // Q / dO pipeline stages
+constexpr int THREADS = 320;
+constexpr int WARP_TMA = 8;
+constexpr int WARP_MMA = 9;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_S = 256, TM_DP = 320, TM_DQ = 384;
+constexpr unsigned FULL = 0xffffffffu;
+
+constexpr uint32_t KV_CHUNK = BN * 128;      // 128 rows x 64 bf16
+constexpr uint32_t KV_TILE = BN * DP * 2;    // 32 KB
+constexpr uint32_t Q_CHUNK = BM * 128;       // 64 rows x 64 bf16
+constexpr uint32_t Q_TILE = BM * DP * 2;     // 16 KB
+constexpr uint32_t DS_TILE = BN * BM * 2;    // 16 KB, 128 rows x 128 B
+
+constexpr uint32_t OFF_K = 0;
+constexpr uint32_t OFF_V = OFF_K + KV_TILE;
+constexpr uint32_t OFF_Q = OFF_V + KV_TILE;
+constexpr uint32_t OFF_DO = OFF_Q + QS * Q_TILE;
+constexpr uint32_t OFF_DS = OFF_DO + QS * Q_TILE;
+constexpr uint32_t OFF_LSE = OFF_DS + 2 * DS_TILE;   // float [QS][BM]: LSE * log2(e)
+constexpr uint32_t OFF_DLT = OFF_LSE + QS * BM * 4;  // float [QS][BM]: D_i
+constexpr uint32_t OFF_BAR = OFF_DLT + QS * BM * 4;
+// kv_full, q_full[QS], q_empty[QS], s_full, p_ready, dp_full, ds_ready,
+// ds_empty[2], dq_full[2], dq_empty[2], dkv_done
+constexpr int NBAR = 1 + 2 * QS + 4 + 2 + 2 + 2 + 1;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory budget");
+
+enum : unsigned {
+  W_KV = 0x20100, W_QEMPTY = 0x20200, W_QFULL = 0x20300, W_SFULL = 0x20400, W_PREADY = 0x20500,
+  W_DPFULL = 0x20600, W_DSREADY = 0x20700, W_DSEMPTY = 0x20800, W_DQFULL = 0x20900,
+  W_DQEMPTY = 0x20a00, W_DKV = 0x20b00
+};
+
+struct Bars {
+  uint32_t b;
+  __device__ uint32_t kv_full() const { return b; }
+  __device__ uint32_t q_full(int s) const { return b + 8u * (1 + s); }
+  __device__ uint32_t q_empty(int s) const { return b + 8u * (1 + QS + s); }
+  __device__ uint32_t s_full() const { return b + 8u * (1 + 2 * QS); }
+  __device__ uint32_t p_ready() const { return b + 8u * (2 + 2 * QS); }
+  __device__ uint32_t dp_full() const { return b + 8u * (3 + 2 * QS); }
+  __device__ uint32_t ds_ready() const { return b + 8u * (4 + 2 * QS); }
+  __device__ uint32_t ds_empty(int i) const { return b + 8u * (5 + 2 * QS + i); }
+  __device__ uint32_t dq_full(int i) const { return b + 8u * (7 + 2 * QS + i); }
+  __device__ uint32_t dq_empty(int i) const { return b + 8u * (9 + 2 * QS + i); }
+  __device__ uint32_t dkv_done() const { return b + 8u * (11 + 2 * QS); }
+};
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DevErr& e,
+                                          volatile int* abort, unsigned where) {
+  const bool ok = mbar_wait(bar, parity, e, abort, where);
+  return __all_sync(FULL, ok);
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+// ------------------------------------------------------------ preprocess ---
+
+// One warp per (token, head) row: D_i = dO_i . O_i into delta [H, T], and the
+// row of the fp32 dQ accumulator set to zero.
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnParams p) {
+  const long long rows = p.total * p.H;
+  const int lane = threadIdx.x % 32;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  for (long long r = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; r < rows; r += warps) {
+    const long long tok = r / p.H;
+    const int h = static_cast<int>(r % p.H);
+    const size_t off = static_cast<size_t>(r) * p.D;
+    const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(p.o) + off;
+    const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(p.dout) + off;
+    float acc = 0.f;
+    for (int d = 2 * lane; d < p.D; d += 64) {
+      const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + d));
+      const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(g + d));
+      acc = fmaf(of.x, gf.x, acc);
+      acc = fmaf(of.y, gf.y, acc);
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(FULL, acc, s);
+    if (lane == 0) p.delta[static_cast<size_t>(h) * p.total + tok] = acc;
+    float4* dq = reinterpret_cast<float4*>(p.dq_accum + off);
+    for (int d4 = lane; d4 < p.D / 4; d4 += 32) dq[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// dQ = bf16(scale * accumulator), 8 elements per thread per iteration.
+__global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const AttnParams p) {
+  const long long n8 = p.total * p.H * p.D / 8;
+  const float4* src = reinterpret_cast<const float4*>(p.dq_accum);
+  uint4* dst = static_cast<uint4*>(p.dq);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = src[2 * i];
+    const float4 b = src[2 * i + 1];
+    uint4 w;
+    w.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
+    w.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
+    w.z = pack_bf16x2(b.x * p.scale, b.y * p.scale);
+    w.w = pack_bf16x2(b.z * p.scale, b.w * p.scale);
+    dst[i] = w;
+  }
+}
+
+// ------------------------------------------------------------------ main ---
+
+__global__ void __launch_bounds__(THREADS, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const AttnParams p, int num_j) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+
+  // Tile order: causal CTAs with the most query tiles (small j) first.
+  const int HB = p.H_kv * p.B;
+  const int j = static_cast<int>(blockIdx.x / HB);
+  const int rem = static_cast<int>(blockIdx.x % HB);
+  const int hk = rem % p.H_kv;
+  const int b = rem / p.H_kv;
+  (void)num_j;
+  const SeqInfo sq = seq_info(p, b);
+  if (!seq_ok(p, sq) || j * BN >= sq.len) return;
+  const int g = p.H / p.H_kv;
+  const int n_q = (sq.len + BM - 1) / BM;
+  const int i0 = p.causal ? (j * BN) / BM : 0;
+  const int n_qt = n_q - i0;         // query tiles per head
+  const int n_steps = g * n_qt;
+
+  const Bars bars{sbase + OFF_BAR};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    *abort = 0;
+    mbar_init(bars.kv_full(), 1);
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(bars.q_full(s), 1);
+      mbar_init(bars.q_empty(s), 1);
+    }
+    mbar_init(bars.s_full(), 1);
+    mbar_init(bars.p_ready(), 128);
+    mbar_init(bars.dp_full(), 1);
+    mbar_init(bars.ds_ready(), 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars.ds_empty(i), 1);
+      mbar_init(bars.dq_full(i), 1);
+      mbar_init(bars.dq_empty(i), 128);
+    }
+    mbar_init(bars.dkv_done(), 1);
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == WARP_TMA) {
+    // ---------------------------------------------------------- producer ---
+    // Lane 0 issues the TMA copies; all 32 lanes stage the step's LSE and D_i
+    // values next to its Q / dO tiles, published by the same q_full barrier.
+    float* s_lse = reinterpret_cast<float*>(smem + OFF_LSE);
+    float* s_dlt = reinterpret_cast<float*>(smem + OFF_DLT);
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      const int row_kv = sq.start + j * BN;
+      mbar_arrive_expect_tx(bars.kv_full(), 2 * KV_TILE);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tma_load_3d(sbase + OFF_K + c * KV_CHUNK, &tm_k, bars.kv_full(), c * 64, hk, row_kv);
+        tma_load_3d(sbase + OFF_V + c * KV_CHUNK, &tm_v, bars.kv_full(), c * 64, hk, row_kv);
+      }
+    }
+    for (int t = 0; t < n_steps; ++t) {
+      const int st = t % QS;
+      const int h = hk * g + t / n_qt;
+      const int qbase = (i0 + t % n_qt) * BM;
+      if (!warp_wait(bars.q_empty(st), ((t / QS) & 1) ^ 1, p.err, abort, W_QEMPTY)) break;
+      for (int q = lane; q < BM; q += 32) {
+        const int qpos = qbase + q;
+        const bool qv = qpos < sq.len;
+        s_lse[st * BM + q] =
+            qv ? p.lse[lse_index(p, b, h, sq.start, qpos)] * 1.4426950408889634f : 0.f;
+        s_dlt[st * BM + q] = qv ? p.delta[static_cast<size_t>(h) * p.total + sq.start + qpos] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const int row_q = sq.start + qbase;
+        mbar_arrive_expect_tx(bars.q_full(st), 2 * Q_TILE);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sbase + OFF_Q + st * Q_TILE + c * Q_CHUNK, &tm_q, bars.q_full(st), c * 64, h,
+                      row_q);
+          tma_load_3d(sbase + OFF_DO + st * Q_TILE + c * Q_CHUNK, &tm_do, bars.q_full(st), c * 64,
+                      h, row_q);
+        }
+      }
+      __syncwarp();
+    }
+    for (int t = max(0, n_steps - QS); t < n_steps && !*abort; ++t)
+      if (!warp_wait(bars.q_empty(t % QS), (t / QS) & 1, p.err, abort, W_QEMPTY)) break;
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      // -------------------------------------------------------- MMA issuer ---
+      constexpr uint32_t ID_SDP = idesc_bf16(BN, BM, false, false);   // S^T, dP^T
+      constexpr uint32_t ID_DVK = idesc_bf16(BN, DP, false, true);    // dV, dK
+      constexpr uint32_t ID_DQ = idesc_bf16(DP, BM, true, true);      // dQ^T
+      bool ok = mbar_wait(bars.kv_full(), 0, p.err, abort, W_KV);
+      for (int t = 0; ok && t <= n_steps; ++t) {
+        if (t < n_steps) {
+          const int st = t % QS;
+          if (!(ok = mbar_wait(bars.q_full(st), (t / QS) & 1, p.err, abort, W_QFULL))) break;
+          tc_fence_after();
+          // S^T = K Q^T
+#pragma unroll
+          for (int kk = 0; kk < DP / 16; ++kk) {
+            const uint32_t ko = (kk >> 2) * KV_CHUNK + (kk & 3) * 32;
+            const uint32_t qo = (kk >> 2) * Q_CHUNK + (kk & 3) * 32;
+            mma_ss(tmem + TM_S, sdesc_sw128(sbase + OFF_K + ko, 16, 1024),
+                   sdesc_sw128(sbase + OFF_Q + st * Q_TILE + qo, 16, 1024), ID_SDP, kk > 0);
+          }
+          tc_commit(bars.s_full());
+          // dP^T = V dO^T, once the softmax warps are done with dP^T of t-1.
+          if (t >= 1 && !(ok = mbar_wait(bars.ds_ready(), (t - 1) & 1, p.err, abort, W_DSREADY)))
+            break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < DP / 16; ++kk) {
+            const uint32_t vo = (kk >> 2) * KV_CHUNK + (kk & 3) * 32;
+            const uint32_t go = (kk >> 2) * Q_CHUNK + (kk & 3) * 32;
+            mma_ss(tmem + TM_DP, sdesc_sw128(sbase + OFF_V + vo, 16, 1024),
+                   sdesc_sw128(sbase + OFF_DO + st * Q_TILE + go, 16, 1024), ID_SDP, kk > 0);
+          }
+          tc_commit(bars.dp_full());
+        }
+        if (t >= 1) {
+          const int u = t - 1;
+          const int su = u % QS;
+          const uint32_t ds = sbase + OFF_DS + (u & 1) * DS_TILE;
+          if (t == n_steps &&
+              !(ok = mbar_wait(bars.ds_ready(), u & 1, p.err, abort, W_DSREADY)))
+            break;
+          tc_fence_after();
+          // dK += dS^T Q   (A: dS^T K-major in smem; B: Q MN-major)
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ss(tmem + TM_DK, sdesc_sw128(ds + kk * 32, 16, 1024),
+                   sdesc_sw128(sbase + OFF_Q + su * Q_TILE + kk * 2048, Q_CHUNK, 1024), ID_DVK,
+                   (u > 0 || kk > 0) ? 1u : 0u);
+          // dQ^T = K^T dS^T  (A: K MN-major; B: dS^T MN-major), into dQ buffer u&1
+          if (!(ok = mbar_wait(bars.dq_empty(u & 1), ((u >> 1) & 1) ^ 1, p.err, abort,
+                               W_DQEMPTY)))
+            break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ss(tmem + TM_DQ + (u & 1) * BM, sdesc_sw128(sbase + OFF_K + kk * 2048, KV_CHUNK, 1024),
+                   sdesc_sw128(ds + kk * 2048, KV_CHUNK, 1024), ID_DQ, kk > 0);
+          tc_commit(bars.dq_full(u & 1));
+          tc_commit(bars.ds_empty(u & 1));
+          tc_commit(bars.q_empty(su));
+        }
+        if (t < n_steps) {
+          const int st = t % QS;
+          if (!(ok = mbar_wait(bars.p_ready(), t & 1, p.err, abort, W_PREADY))) break;
+          tc_fence_after();
+          // dV += P^T dO  (A: P^T from TMEM; B: dO MN-major)
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8,
+                   sdesc_sw128(sbase + OFF_DO + st * Q_TILE + kk * 2048, Q_CHUNK, 1024), ID_DVK,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      tc_commit(bars.dkv_done());
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------- softmax / dS warps ---
+    const int r = threadIdx.x;            // key row in the tile = TMEM lane
+    const int kpos = j * BN + r;          // key position in the sequence
+    const bool key_ok = kpos < sq.len;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    float* s_lse = reinterpret_cast<float*>(smem + OFF_LSE);
+    float* s_dlt = reinterpret_cast<float*>(smem + OFF_DLT);
+    const float c2 = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < n_steps && ok; ++t) {
+      const int h = hk * g + t / n_qt;
+      const int qbase = (i0 + t % n_qt) * BM;   // first query of the tile
+      const int st = t % QS;
+      const float* lse_t = s_lse + st * BM;
+      const float* dlt_t = s_dlt + st * BM;
+      (void)h;
+      // The stage's LSE / D_i values (and Q, dO) have landed.
+      if (!(ok = warp_wait(bars.q_full(st), (t / QS) & 1, p.err, abort, W_QFULL))) break;
+      // Visible queries of this key row: qpos in [qlo, qhi).
+      const int qlo = p.causal ? kpos : 0;
+      const int qhi = key_ok ? sq.len : 0;
+
+      if (!(ok = warp_wait(bars.s_full(), t & 1, p.err, abort, W_SFULL))) break;
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(tmem + lane_off + TM_S, sr[0]);
+      tmem_ld32(tmem + lane_off + TM_S + 32, sr[1]);
+      tmem_ld_wait();
+      reg_fence(sr[0]);
+      reg_fence(sr[1]);
+      float pr[BM];
+      uint32_t pk[32];
+#pragma unroll
+      for (int q = 0; q < BM; q += 2) {
+        const int qp = qbase + q;
+        const float s0 = __uint_as_float(sr[q >> 5][q & 31]);
+        const float s1 = __uint_as_float(sr[q >> 5][(q + 1) & 31]);
+        const float p0 = (qp >= qlo && qp < qhi) ? ex2_approx(fmaf(s0, c2, -lse_t[q])) : 0.f;
+        const float p1 = (qp + 1 >= qlo && qp + 1 < qhi) ? ex2_approx(fmaf(s1, c2, -lse_t[q + 1]))
+                                                        : 0.f;
+        pr[q] = p0;
+        pr[q + 1] = p1;
+        pk[q >> 1] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(tmem + lane_off + TM_S, pk);   // P^T (bf16) over S^T
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bars.p_ready());
+
+      if (!(ok = warp_wait(bars.dp_full(), t & 1, p.err, abort, W_DPFULL))) break;
+      tc_fence_after();
+      uint32_t dr[2][32];
+      tmem_ld32(tmem + lane_off + TM_DP, dr[0]);
+      tmem_ld32(tmem + lane_off + TM_DP + 32, dr[1]);
+      tmem_ld_wait();
+      reg_fence(dr[0]);
+      reg_fence(dr[1]);
+      // dS^T row into the shared buffer t&1 once the MMAs of step t-2 are done.
+      if (!(ok = warp_wait(bars.ds_empty(t & 1), ((t >> 1) & 1) ^ 1, p.err, abort, W_DSEMPTY)))
+        break;
+      uint8_t* ds_row = smem + OFF_DS + (t & 1) * DS_TILE + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {   // 16-byte chunk c holds queries 8c..8c+7
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int q = 8 * c + 2 * e;
+          const float d0 = pr[q] * (__uint_as_float(dr[q >> 5][q & 31]) - dlt_t[q]);
+          const float d1 = pr[q + 1] * (__uint_as_float(dr[q >> 5][(q + 1) & 31]) - dlt_t[q + 1]);
+          w[e] = pack_bf16x2(d0, d1);
+        }
+        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars.ds_ready());
+    }
+    // ---------------------------------------------------- dK / dV epilogue ---
+    if (ok && warp_wait(bars.dkv_done(), 0, p.err, abort, W_DKV)) {
+      tc_fence_after();
+      const bool store = key_ok;
+      const size_t off = (static_cast<size_t>(sq.start + kpos) * p.H_kv + hk) * p.D;
+      __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + off;
+      __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + off;
+#pragma unroll
+      for (int c = 0; c < DP / 32; ++c) {
+        uint32_t a[32], v[32];
+        tmem_ld32(tmem + lane_off + TM_DK + 32 * c, a);
+        tmem_ld32(tmem + lane_off + TM_DV + 32 * c, v);
+        tmem_ld_wait();
+        reg_fence(a);
+        reg_fence(v);
+        if (store && 32 * c < p.D) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 wk, wv;
+            uint32_t* pk4 = &wk.x;
+            uint32_t* pv4 = &wv.x;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 8 * v4 + 2 * e;
+              pk4[e] = pack_bf16x2(__uint_as_float(a[i]) * p.scale,
+                                   __uint_as_float(a[i + 1]) * p.scale);
+              pv4[e] = pack_bf16x2(__uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+            }
+            reinterpret_cast<uint4*>(dk + 32 * c)[v4] = wk;
+            reinterpret_cast<uint4*>(dv + 32 * c)[v4] = wv;
+          }
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------ dQ drain warps ---
+    const int d = (warp - 4) * 32 + lane;     // head-dim row of dQ^T = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    for (int u = 0; u < n_steps; ++u) {
+      if (!warp_wait(bars.dq_full(u & 1), (u >> 1) & 1, p.err, abort, W_DQFULL)) break;
+      tc_fence_after();
+      uint32_t qr[2][32];
+      tmem_ld32(tmem + lane_off + TM_DQ + (u & 1) * BM, qr[0]);
+      tmem_ld32(tmem + lane_off + TM_DQ + (u & 1) * BM + 32, qr[1]);
+      tmem_ld_wait();
+      reg_fence(qr[0]);
+      reg_fence(qr[1]);
+      tc_fence_before();
+      mbar_arrive(bars.dq_empty(u & 1));
+      const int h = hk * g + u / n_qt;
+      const int qbase = (i0 + u % n_qt) * BM;
+      if (d < p.D) {
+        const int qn = min(BM, sq.len - qbase);
+        float* dst = p.dq_accum + (static_cast<size_t>(sq.start + qbase) * p.H + h) * p.D + d;
+        const size_t stride = static_cast<size_t>(p.H) * p.D;
+#pragma unroll
+        for (int q = 0; q < BM; ++q)
+          if (q < qn) red_add_f32(dst + q * stride, __uint_as_float(qr[q >> 5][q & 31]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned mask) {
+  if (p.D != 64 && p.D != 128) return cudaErrorInvalidValue;
+  if (p.total == 0) return cudaSuccess;
+  const long long rows = p.total * p.H;
+  cudaError_t e = cudaSuccess;
+  if (mask & 1u) {
+    const int pre_blocks = static_cast<int>(std::min<long long>((rows + 7) / 8, 148LL * 16));
+    bwd_preprocess_kernel<<<pre_blocks, 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (!(mask & 2u)) goto convert;
+  {
+
+  const int num_j = (p.max_seqlen + BN - 1) / BN;
+  const long long tiles = static_cast<long long>(num_j) * p.H_kv * p.B;
+  if (tiles > INT_MAX) return cudaErrorInvalidConfiguration;
+  if (tiles > 0) {
+    CUtensorMap tq, tk, tv, tg;
+    if (!make_tmap_bf16_3d(&tq, p.q, p.total, p.H, p.D, BM) ||
+        !make_tmap_bf16_3d(&tk, p.k, p.total, p.H_kv, p.D, BN) ||
+        !make_tmap_bf16_3d(&tv, p.v, p.total, p.H_kv, p.D, BN) ||
+        !make_tmap_bf16_3d(&tg, p.dout, p.total, p.H, p.D, BM))
+      return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    bwd_main_kernel<<<static_cast<unsigned>(tiles), THREADS, SMEM, stream>>>(tq, tk, tv, tg, p,
+                                                                           num_j);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  }
+convert:
+  if (mask & 4u) {
+    const long long n8 = rows * p.D / 8;
+    const int cv_blocks = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148LL * 16));
+    bwd_dq_convert_kernel<<<cv_blocks, 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+  }
+  return e;
+}
 
 }  // namespace fa

@@ -114,6 +114,21 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long ro
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
+                       unsigned box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(heads) * D * 2};
+  const cuuint32_t box[3] = {64, 1, box_rows};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
 __global__ void wait_selftest_kernel(DevErr e) {
@@ -178,6 +193,17 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int D, fa_dtype dtype, int causal, float scale, const int* cu_seqlens,
                  int max_seqlen, long long total_tokens, void* workspace, size_t ws_bytes,
                  fa_stream_t stream) {
+  return fa_bwd_phases(7u, q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, D, dtype, causal,
+                       scale, cu_seqlens, max_seqlen, total_tokens, workspace, ws_bytes, stream);
+}
+
+fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void* v,
+                        const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                        void* dv, int B, int H, int H_kv, int N, int D, fa_dtype dtype, int causal,
+                        float scale, const int* cu_seqlens, int max_seqlen, long long total_tokens,
+                        void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  if (mask == 0 || mask > 7u) return FA_ERR_INVALID_ARG;
+  if (dtype == FA_F32 && mask != 7u) return FA_ERR_UNSUPPORTED;
   AttnParams p = {};
   fa_status st = fa::check_common(p, B, H, H_kv, N, D, dtype, causal, scale, cu_seqlens,
                                   max_seqlen, total_tokens);
@@ -209,7 +235,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.err.word = fa::err_word();
   if (p.err.word == nullptr) return FA_ERR_CUDA;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e = (dtype == FA_F32) ? fa::launch_bwd_f32(p, s) : fa::launch_bwd_bf16(p, s);
+  const cudaError_t e =
+      (dtype == FA_F32) ? fa::launch_bwd_f32(p, s) : fa::launch_bwd_bf16(p, s, mask);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -70,7 +70,8 @@ __device__ __forceinline__ size_t lse_index(const AttnParams& p, int b, int h, i
 cudaError_t launch_fwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream);
-cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream);
+// mask: bit 0 preprocess, bit 1 main kernel, bit 2 dQ conversion.
+cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned mask);
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
 
 // Host: cuTensorMapEncodeTiled through the runtime's driver entry point.
@@ -78,5 +79,11 @@ cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
 // box of box_cols x box_rows and 128-byte swizzle. Returns false on failure.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long rows,
                        unsigned long long cols, unsigned box_cols, unsigned box_rows);
+
+// Host: 3-D bf16 view (D, heads, rows) of a token-major [rows, heads, D]
+// tensor with a (64, 1, box_rows) box and 128-byte swizzle. Column blocks at
+// x >= D lie outside the tensor and arrive as zeros.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
+                       unsigned box_rows);
 
 }  // namespace fa

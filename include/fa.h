@@ -140,6 +140,21 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int max_seqlen, long long total_tokens, void* workspace, size_t ws_bytes,
                  fa_stream_t stream);
 
+/*
+ * fa_bwd_phases - fa_bwd restricted to some of its three kernels, so that
+ * each can be timed by itself: bit 0 = preprocess (D_i = dO_i . O_i and
+ * zeroing of the fp32 dQ accumulator), bit 1 = the main tensor-core kernel
+ * (recomputation, dK, dV and accumulation of dQ), bit 2 = conversion of the
+ * accumulator to dQ. fa_bwd(...) is fa_bwd_phases(7, ...). Phases must be
+ * enqueued in that order on the same workspace. For FA_F32 only mask 7 is
+ * accepted (FA_ERR_UNSUPPORTED otherwise). Other arguments as for fa_bwd.
+ */
+fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void* v,
+                        const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                        void* dv, int B, int H, int H_kv, int N, int D, fa_dtype dtype, int causal,
+                        float scale, const int* cu_seqlens, int max_seqlen, long long total_tokens,
+                        void* workspace, size_t ws_bytes, fa_stream_t stream);
+
 /* fa_get_error_string - static, human-readable name of a status code. */
 const char* fa_get_error_string(fa_status status);
 

@@ -63,3 +63,85 @@ def test_f32_varlen_ragged(causal):
     lengths = [1, 0, 45, 130, 3]
     inp = random_case(8, dtype="f32", lengths=lengths, H=4, H_kv=2, D=64, varlen=True)
     check_f32(inp, causal, 0.125, len(lengths), 0)
+
+
+# --------------------------------------------------------------- bf16 path ---
+
+def check_bf16(inp, causal, scale, B, N):
+    got = run_fwd_bwd(inp, causal, scale, B, N)
+    ref = oa.attention_backward(inp.q, inp.k, inp.v, inp.do, inp.cu_seqlens.numpy(), causal, scale)
+    for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
+        assert np.isfinite(g).all(), name
+        err = rel_fro(g, r)
+        assert err <= REL_BF16, f"{name} rel-Frobenius {err}"
+
+
+BWD_CASES = [
+    # (B, N, H, H_kv, D)
+    (1, 128, 2, 2, 128),
+    (2, 300, 4, 2, 128),
+    (1, 1, 2, 1, 128),
+    (1, 65, 2, 2, 128),
+    (1, 200, 2, 2, 64),
+    (2, 129, 3, 1, 64),
+    (1, 513, 4, 1, 128),
+]
+
+
+@pytest.mark.parametrize("B,N,H,H_kv,D", BWD_CASES)
+@pytest.mark.parametrize("causal", [False, True])
+def test_bf16_dense(B, N, H, H_kv, D, causal):
+    inp = random_case(B * 1000 + N + D + 7, dtype="bf16", lengths=[N] * B, H=H, H_kv=H_kv, D=D,
+                      varlen=False)
+    check_bf16(inp, causal, D ** -0.5, B, N)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bf16_varlen_ragged(D, causal):
+    lengths = [5, 0, 128, 1, 300, 129, 64]
+    inp = random_case(78, dtype="bf16", lengths=lengths, H=4, H_kv=2, D=D, varlen=True)
+    check_bf16(inp, causal, D ** -0.5, len(lengths), 0)
+
+
+def test_bf16_large_logits():
+    inp = random_case(3, dtype="bf16", lengths=[384], H=2, H_kv=2, D=128, varlen=False, std=2.8)
+    for causal in (False, True):
+        check_bf16(inp, causal, 128 ** -0.5, 1, 384)
+
+
+@pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items()
+                                  if w.dtype == "bf16" and w.backward])
+def test_bf16_workload_group_slice(name):
+    """Full-size workload; one key/value head group of one sequence checked."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    B = len(inp.cu_seqlens) - 1
+    a = to_api(inp, B, w.N)
+    kw = dict(causal=w.causal, scale=w.scale, cu_seqlens=a.get("cu_seqlens"),
+              max_seqlen=a.get("max_seqlen"))
+    o, lse = fa.fwd(a["q"], a["k"], a["v"], **kw)
+    dq, dk, dv = fa.bwd(a["do"], a["q"], a["k"], a["v"], o, lse, **kw)
+    st, where = fa.check_device_error()
+    assert st == 0, f"device error {st} at {where:#x}"
+    T = inp.q.shape[0]
+    dq = dq.reshape(T, w.H, w.D)
+    dk = dk.reshape(T, w.H_kv, w.D)
+    dv = dv.reshape(T, w.H_kv, w.D)
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t).all()
+    cu = inp.cu_seqlens.tolist()
+    b = int(np.argmax(np.diff(cu)))   # the longest sequence
+    hk = w.H_kv - 1
+    s0, s1 = cu[b], cu[b + 1]
+    g = w.H // w.H_kv
+    ref_dk = np.zeros((s1 - s0, w.D))
+    ref_dv = np.zeros((s1 - s0, w.D))
+    for h in range(hk * g, (hk + 1) * g):
+        rdq, rdk, rdv = oa.head_backward(inp.q[s0:s1, h], inp.k[s0:s1, hk], inp.v[s0:s1, hk],
+                                         inp.do[s0:s1, h], w.scale, w.causal)
+        assert rel_fro(f64(dq[s0:s1, h]), rdq) <= REL_BF16
+        ref_dk += rdk
+        ref_dv += rdv
+    assert rel_fro(f64(dk[s0:s1, hk]), ref_dk) <= REL_BF16
+    assert rel_fro(f64(dv[s0:s1, hk]), ref_dv) <= REL_BF16
