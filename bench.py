@@ -1,0 +1,433 @@
+#!/usr/bin/env python3
+"""Attention forward + backward throughput on B200, one JSON line.
+
+A step is one pass of the whole hot path over one batch of the workload:
+fa_fwd (O, LSE) then fa_bwd (preprocess, fused dK/dV/dQ kernel, dQ
+conversion), all through the C ABI of libfa_b200.so. Inputs are seeded
+synthetic Gaussians resident in HBM before the timed region starts.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the float64 CPU oracle arm)
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+independently seeded batch of the same shape (the (batch, head) units are
+independent; no collective on the data path): weak scaling, timed as the
+max over ranks of CUDA-event time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16, device-timed) and % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "bf16_causal_b2_h16_n8192_d128"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ host logic ---
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def step_flops(lengths, H: int, D: int, causal: bool) -> tuple:
+    """Algorithmic FLOPs: forward 4*H*sum(L^2)*D, backward 2.5x, causal halves."""
+    from exact_io_aware_tmem_b200.workloads import flops
+    return flops(lengths, H, D, causal)
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch: same shape, independent values."""
+    return seed + 1000 * rank
+
+
+def aggregate(units_per_rank: float, world: int, times_s: list) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / max(times_s)
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max over ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def source_sha(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "exact_io_aware_tmem_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "bwd_main_kernel": ("bwd_bf16.cu", "common.cuh", "params.h")}
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("workload") != workload or rec.get("source_sha") != source_sha(*KERNEL_SOURCES[kernel]):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.strip()]
+        os.unlink(self.out.name)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[0]))
+                smax.append(float(r[1]))
+                power.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- oracle ---
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, n_tokens: int):
+    """Forward + backward of one query head of the workload, truncated to
+    ``n_tokens`` positions, with the float64 oracle. Returns (seconds, flops)."""
+    import torch
+    from exact_io_aware_tmem_b200.workloads import random_case
+    from oracle import attention as oa
+    inp = random_case(w.seed, dtype=w.dtype, lengths=[n_tokens], H=1, H_kv=1, D=w.D, varlen=False,
+                      std=w.qk_mult)
+    q = inp.q[:, 0].to(torch.float64).numpy()
+    k = inp.k[:, 0].to(torch.float64).numpy()
+    v = inp.v[:, 0].to(torch.float64).numpy()
+    do = inp.do[:, 0].to(torch.float64).numpy()
+    t0 = time.perf_counter()
+    oa.head_forward(q, k, v, w.scale, w.causal)
+    oa.head_backward(q, k, v, do, w.scale, w.causal)
+    dt = time.perf_counter() - t0
+    fwd, bwd = step_flops([n_tokens], 1, w.D, w.causal)
+    return dt, fwd + bwd
+
+
+def oracle_tokens_for(w, seconds: float) -> int:
+    """Sequence length of the oracle sample that takes about ``seconds``."""
+    n0 = 512
+    t0, _ = oracle_sample(w, n0)
+    n = int(n0 * math.sqrt(max(seconds, 0.05) / max(t0, 1e-3)))
+    n = max(128, min(w.N, n // 128 * 128))
+    return n
+
+
+def cpu_baseline(w, seconds: float = 15.0) -> dict:
+    n = oracle_tokens_for(w, seconds)
+    dt, fl = oracle_sample(w, n)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "seconds": round(dt, 3),
+            "sample": f"float64 numpy oracle, forward+backward of one query head of "
+                      f"{w.name} truncated to N={n} (causal={w.causal}, D={w.D}); FLOPs by the "
+                      f"same formula as the GPU line"}
+
+
+def run_reference(args, w) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    n = oracle_tokens_for(w, per_step)
+    for _ in range(args.warmup):
+        oracle_sample(w, n)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(w, n)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"float64 numpy oracle, one query head of {w.name} truncated to N={n}, "
+              f"forward+backward per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w) -> dict:
+    from exact_io_aware_tmem_b200.workloads import make_inputs  # noqa: F401
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "D": w.D,
+            "causal": w.causal, "varlen": w.varlen is not None, "pass": "fwd+bwd",
+            "seed": w.seed}
+
+
+# -------------------------------------------------------------- GPU arm ---
+
+def run_ours(args, w) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import exact_io_aware_tmem_b200 as fa
+    from exact_io_aware_tmem_b200.workloads import Workload, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    peaks = load_peaks()
+
+    # Baseline on the host first (rank 0, one GPU only), before any GPU work.
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    wr = Workload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})
+    inp = make_inputs(wr)
+    B = len(inp.cu_seqlens) - 1
+    lengths = inp.cu_seqlens.diff().tolist()
+    fwd_fl, bwd_fl = step_flops(lengths, w.H, w.D, w.causal)
+    T = inp.q.shape[0]
+
+    def to_dev(t):
+        t = t.to(dev)
+        return t if inp.varlen else t.view(B, w.N, t.shape[1], w.D)
+
+    q, k, v, do = (to_dev(t) for t in (inp.q, inp.k, inp.v, inp.do))
+    kw = dict(causal=w.causal, scale=w.scale)
+    if inp.varlen:
+        kw.update(cu_seqlens=inp.cu_seqlens.to(dev), max_seqlen=inp.max_seqlen)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, w.H, w.N) if not inp.varlen else (w.H, T), device=dev,
+                      dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.workspace_size(T, w.H, w.D, q.dtype), dtype=torch.uint8, device=dev)
+    bytes_in = sum(t.numel() * t.element_size() for t in (q, k, v, do))
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        fa.fwd(q, k, v, out=o, lse=lse, **kw)
+        if ev is not None:
+            ev[1].record()
+        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=1, **kw)
+        if ev is not None:
+            ev[2].record()
+        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=2, **kw)
+        if ev is not None:
+            ev[3].record()
+        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=4, **kw)
+        if ev is not None:
+            ev[4].record()
+
+    for _ in range(args.warmup):
+        step()
+    st, where = fa.check_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where:#x} during warm-up")
+
+    gpu_uuid = ""
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        gpu_uuid = gpu_uuid if gpu_uuid.startswith("GPU-") else "GPU-" + gpu_uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_uuid)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    start.record()
+    for i in range(args.steps):
+        step(evs[i])
+    end.record()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    st, where = fa.check_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where:#x} in the timed region")
+    elapsed_ms = start.elapsed_time(end)
+    max_ms = reduce_max(elapsed_ms, dev)
+    k_ms = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+            for name, (a, b) in {"fwd_bf16_kernel": (0, 1), "bwd_preprocess": (1, 2),
+                                 "bwd_main_kernel": (2, 3), "bwd_dq_convert": (3, 4)}.items()}
+    k_ms = {n: reduce_max(t, dev) for n, t in k_ms.items()}
+
+    # End to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, forward + backward, D2H of every output.
+    e2e_steps = max(3, min(args.steps, 20))
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    outs = (o, lse, dq, dk, dv)
+    houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    bytes_out = sum(t.numel() * t.element_size() for t in outs)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record()
+    for _ in range(e2e_steps):
+        for dst, src in zip((q, k, v, do), (hq, hk, hv, hdo)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(houts, outs):
+            dst.copy_(src, non_blocking=True)
+    e_end.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e_start.elapsed_time(e_end), dev)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    per_step_fl = fwd_fl + bwd_fl
+    value = aggregate(per_step_fl * args.steps, world, [max_ms / 1e3]) / 1e12
+    fwd_tf = fwd_fl / (k_ms["fwd_bf16_kernel"] / 1e3) / 1e12
+    bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_main_kernel"] + k_ms["bwd_dq_convert"]
+    bwd_tf = bwd_fl / (bwd_ms / 1e3) / 1e12
+    # Dominant kernel: the one with the larger share of the step.
+    dom = max(("fwd_bf16_kernel", "bwd_main_kernel"), key=lambda n: k_ms[n])
+    dom_fl = fwd_fl if dom == "fwd_bf16_kernel" else bwd_fl
+    achieved = dom_fl / (k_ms[dom] / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(w), parallelism=f"replicas{world}" if world > 1 else "none",
+                       l2=f"not flushed: every step reads and writes "
+                          f"{(bytes_in + bytes_out) / 2**20:.0f} MiB > {L2_BYTES >> 20} MiB L2",
+                       ranks="each rank its own seeded batch of this shape"),
+        "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+        "fwd_frac_of_peak": fwd_tf / peaks["bf16_tflops"],
+        "bwd_frac_of_peak": bwd_tf / peaks["bf16_tflops"],
+        "peak_tflops": {"burst": peaks["bf16_tflops"], "sustained": peaks["bf16_tflops_sustained"],
+                        "source": peaks["source"]},
+        "kernel_ms": {n: round(t, 4) for n, t in k_ms.items()},
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_kind": f"{peaks['source']} sustained bf16",
+                     "traffic": recorded_traffic(dom, w.name)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": per_step_fl * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                "steps": e2e_steps, "h2d_bytes_per_step": bytes_in,
+                "d2h_bytes_per_step": bytes_out},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    from exact_io_aware_tmem_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
