@@ -136,25 +136,30 @@ class ClockSampler:
             self.proc.kill()
         self.out.flush()
         self.out.seek(0)
-        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.strip()]
+        text = self.out.read()
         os.unlink(self.out.name)
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            r = [x.strip() for x in r]
-            try:
-                sm.append(float(r[0]))
-                smax.append(float(r[1]))
-                power.append(float(r[2]))
-            except (ValueError, IndexError):
-                continue
-            for n, v in zip(names, r[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(power) if power else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return parse_clock_rows(text)
+
+
+def parse_clock_rows(text: str) -> dict:
+    """Median SM clock, max clock and the throttle reasons seen in the samples."""
+    sm, smax, power, reasons = [], [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in text.strip().splitlines():
+        r = [x.strip() for x in line.split(",")]
+        try:
+            sm.append(float(r[0]))
+            smax.append(float(r[1]))
+            power.append(float(r[2]))
+        except (ValueError, IndexError):
+            continue
+        for n, v in zip(names, r[3:7]):
+            if v.lower() == "active":
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "power_w_max": max(power) if power else None,
+            "samples": len(sm), "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------- oracle ---
