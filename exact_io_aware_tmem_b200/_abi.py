@@ -37,6 +37,9 @@ SIGNATURES = {
                               c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
                               c_int, c_int, c_int, c_float, c_void_p, c_int, c_ll, c_void_p,
                               c_size_t, c_void_p]),
+    "fa_bwd_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                               c_int, c_int, c_float, c_void_p, c_int, c_ll, c_void_p]),
     "fa_get_error_string": (ctypes.c_char_p, [c_int]),
     "fa_check_device_error": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_uint)]),
     "fa_set_wait_budget": (None, [c_ll]),

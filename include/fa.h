@@ -155,6 +155,39 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
                         float scale, const int* cu_seqlens, int max_seqlen, long long total_tokens,
                         void* workspace, size_t ws_bytes, fa_stream_t stream);
 
+/*
+ * fa_bwd_noalloc - fa_bwd for callers that cannot allocate device memory.
+ *
+ * The pages describe no such call; it exists for callers that are handed only
+ * their input and output buffers and may not call cudaMalloc themselves (a
+ * kernel plugin inside a framework that owns every device allocation, or a
+ * latency-critical path where an allocation would synchronise the device or
+ * break a fixed memory budget). Instead of a caller workspace it uses a
+ * scratch array built into the library: FA_NOALLOC_SCRATCH_BYTES (32 MiB) of
+ * device memory that every GPU loading the library holds until the process
+ * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments, layouts and results are those of fa_bwd without workspace and
+ * ws_bytes. Limit: fa_bwd_workspace_size(T, H, D, dtype) must not exceed
+ * FA_NOALLOC_SCRATCH_BYTES (for bf16 about T * H * (D + 1) * 4 bytes, e.g.
+ * T * H <= 64000 at D = 128); larger problems return FA_ERR_UNSUPPORTED
+ * before anything is enqueued.
+ *
+ * The scratch is shared by every call on a device and keeps the last call's
+ * contents; each call re-initialises what it reads. Calls whose kernels can
+ * overlap on the GPU (different streams without ordering between them, or
+ * several host threads) race on the scratch and give wrong results: order
+ * them on one stream. The first call on each device looks up the scratch's
+ * device address (cudaGetSymbolAddress) once, with that device current; make
+ * that first call before any stream capture begins.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                         int H, int H_kv, int N, int D, fa_dtype dtype, int causal, float scale,
+                         const int* cu_seqlens, int max_seqlen, long long total_tokens,
+                         fa_stream_t stream);
+
 /* fa_get_error_string - static, human-readable name of a status code. */
 const char* fa_get_error_string(fa_status status);
 
