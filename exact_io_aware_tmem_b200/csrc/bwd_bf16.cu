@@ -23,15 +23,16 @@
 //                      dS^T = P^T * (dP^T - D_i)  -> bf16 in shared memory
 //                      dK  += dS^T Q_i
 //                      dQ_i^T = K_j^T dS^T           (M=128 = D lanes, N=64)
-//                    and the dQ^T tile is added into the fp32 accumulator
-//                    by per-element red.global.add.f32 (the separate
-//                    dQ-accumulation path); dK, dV are scaled and stored at
-//                    the end.
+//                    and the dQ^T tile is staged in shared memory and added
+//                    into the fp32 accumulator with one TMA bulk reduce-add
+//                    per step (the separate dQ-accumulation path); dK, dV
+//                    are scaled and stored at the end.
 //   bwd_dq_convert   dQ = bf16(scale * accumulator).
 //
-// Roles in bwd_main (320 threads): warps 0-3 softmax / dS (thread = key row
-// = TMEM lane) and the dK/dV epilogue; warps 4-7 dQ drain (thread = head-dim
-// row of dQ^T); warp 8 TMA producer; warp 9 MMA issuer.
+// Roles in bwd_main (448 threads): warps 0-7 softmax / dS and the dK/dV
+// epilogue (thread = key row = TMEM lane, warps w and w+4 split the 64 query
+// columns); warps 8-11 dQ drain (thread = head-dim row of dQ^T); warp 12 TMA
+// producer; warp 13 MMA issuer.
 // TMEM columns: dV [0,128) dK [128,256) S/P [256,320) dP [320,384)
 //               dQ^T x2 [384,512).
 // D = 64 runs the same kernel: the tensor maps are 3-D (D, heads, tokens), so
@@ -49,10 +50,12 @@ namespace {
 constexpr int BN = 128;  // keys per CTA (TMEM lanes)
 constexpr int BM = 64;   // query rows per step
 constexpr int DP = 128;  // padded head dim
-constexpr int QS = 2;    // Q / dO pipeline stages
-constexpr int THREADS = 320;
-constexpr int WARP_TMA = 8;
-constexpr int WARP_MMA = 9;
+constexpr int QS = 3;    // Q / dO pipeline stages
+constexpr int THREADS = 448;
+constexpr int WARP_DQ0 = 8;    // first of the four dQ drain warps
+constexpr int WARP_TMA = 12;
+constexpr int WARP_MMA = 13;
+constexpr int N_SOFTMAX = 256; // threads in warps 0-7
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_S = 256, TM_DP = 320, TM_DQ = 384;
 constexpr unsigned FULL = 0xffffffffu;
@@ -62,26 +65,31 @@ constexpr uint32_t KV_TILE = BN * DP * 2;    // 32 KB
 constexpr uint32_t Q_CHUNK = BM * 128;       // 64 rows x 64 bf16
 constexpr uint32_t Q_TILE = BM * DP * 2;     // 16 KB
 constexpr uint32_t DS_TILE = BN * BM * 2;    // 16 KB, 128 rows x 128 B
+constexpr uint32_t DQ_STAGE = BM * DP * 4;   // 32 KB, fp32 [64 queries][D]
 
 constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = OFF_K + KV_TILE;
 constexpr uint32_t OFF_Q = OFF_V + KV_TILE;
 constexpr uint32_t OFF_DO = OFF_Q + QS * Q_TILE;
 constexpr uint32_t OFF_DS = OFF_DO + QS * Q_TILE;
-constexpr uint32_t OFF_LSE = OFF_DS + 2 * DS_TILE;   // float [QS][BM]: LSE * log2(e)
+constexpr uint32_t OFF_DQS = OFF_DS + 2 * DS_TILE;  // dQ tile staged for the bulk reduce
+constexpr uint32_t OFF_LSE = OFF_DQS + DQ_STAGE;     // float [QS][BM]: LSE * log2(e)
 constexpr uint32_t OFF_DLT = OFF_LSE + QS * BM * 4;  // float [QS][BM]: D_i
 constexpr uint32_t OFF_BAR = OFF_DLT + QS * BM * 4;
 // kv_full, q_full[QS], q_empty[QS], s_full, p_ready, dp_full, ds_ready,
-// ds_empty[2], dq_full[2], dq_empty[2], dkv_done
-constexpr int NBAR = 1 + 2 * QS + 4 + 2 + 2 + 2 + 1;
+// ds_empty[2], dq_full[2], dq_empty[2], dkv_done, dq_staged, dq_sfree
+constexpr int NBAR = 1 + 2 * QS + 4 + 2 + 2 + 2 + 1 + 2;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;
+// No alignment slack: the layout only fits if the dynamic shared memory
+// starts on a 1024-byte boundary (the 128-byte swizzle atoms need it). The
+// kernel checks this at run time and reports instead of running misaligned.
+constexpr uint32_t SMEM = OFF_MISC + 16;
 static_assert(SMEM <= 232448, "shared memory budget");
 
 enum : unsigned {
   W_KV = 0x20100, W_QEMPTY = 0x20200, W_QFULL = 0x20300, W_SFULL = 0x20400, W_PREADY = 0x20500,
   W_DPFULL = 0x20600, W_DSREADY = 0x20700, W_DSEMPTY = 0x20800, W_DQFULL = 0x20900,
-  W_DQEMPTY = 0x20a00, W_DKV = 0x20b00
+  W_DQEMPTY = 0x20a00, W_DKV = 0x20b00, W_DQSTAGED = 0x20c00, W_DQSFREE = 0x20d00
 };
 
 struct Bars {
@@ -97,6 +105,8 @@ struct Bars {
   __device__ uint32_t dq_full(int i) const { return b + 8u * (7 + 2 * QS + i); }
   __device__ uint32_t dq_empty(int i) const { return b + 8u * (9 + 2 * QS + i); }
   __device__ uint32_t dkv_done() const { return b + 8u * (11 + 2 * QS); }
+  __device__ uint32_t dq_staged() const { return b + 8u * (12 + 2 * QS); }
+  __device__ uint32_t dq_sfree() const { return b + 8u * (13 + 2 * QS); }
 };
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DevErr& e,
@@ -118,8 +128,26 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+// Element-wise add of a shared-memory tile into global memory by the TMA
+// unit (no multicast), tracked as a bulk async-group of this thread.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int x,
+                                                  int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until this thread's bulk groups have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Wait until this thread's bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ------------------------------------------------------------ preprocess ---
@@ -175,11 +203,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_do, const AttnParams p, int num_j) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+                    const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dq, const AttnParams p, int num_j) {
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
+  if ((sbase & 1023u) != 0) {
+    if (threadIdx.x == 0) {
+      atomicOr(p.err.word, ERR_BOUNDS);
+      atomicExch(p.err.word + 1, 0x20A11Bu);
+    }
+    return;
+  }
 
   // Tile order: causal CTAs with the most query tiles (small j) first.
   const int HB = p.H_kv * p.B;
@@ -206,19 +240,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort = 0;
     mbar_init(bars.kv_full(), 1);
     for (int s = 0; s < QS; ++s) {
-      mbar_init(bars.q_full(s), 1);
+      mbar_init(bars.q_full(s), 2);  // TMA bytes + staged LSE / D_i
       mbar_init(bars.q_empty(s), 1);
     }
     mbar_init(bars.s_full(), 1);
-    mbar_init(bars.p_ready(), 128);
+    mbar_init(bars.p_ready(), N_SOFTMAX);
     mbar_init(bars.dp_full(), 1);
-    mbar_init(bars.ds_ready(), 128);
+    mbar_init(bars.ds_ready(), N_SOFTMAX);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.ds_empty(i), 1);
       mbar_init(bars.dq_full(i), 1);
       mbar_init(bars.dq_empty(i), 128);
     }
     mbar_init(bars.dkv_done(), 1);
+    mbar_init(bars.dq_staged(), 128);
+    mbar_init(bars.dq_sfree(), 1);
     fence_mbar_init();
   }
   if (warp == WARP_MMA) {
@@ -241,6 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_dq);
       const int row_kv = sq.start + j * BN;
       mbar_arrive_expect_tx(bars.kv_full(), 2 * KV_TILE);
 #pragma unroll
@@ -254,15 +291,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int h = hk * g + t / n_qt;
       const int qbase = (i0 + t % n_qt) * BM;
       if (!warp_wait(bars.q_empty(st), ((t / QS) & 1) ^ 1, p.err, abort, W_QEMPTY)) break;
-      for (int q = lane; q < BM; q += 32) {
-        const int qpos = qbase + q;
-        const bool qv = qpos < sq.len;
-        s_lse[st * BM + q] =
-            qv ? p.lse[lse_index(p, b, h, sq.start, qpos)] * 1.4426950408889634f : 0.f;
-        s_dlt[st * BM + q] = qv ? p.delta[static_cast<size_t>(h) * p.total + sq.start + qpos] : 0.f;
-      }
-      __syncwarp();
       if (lane == 0) {
+        // Tiles first, so the copies overlap the LSE / D_i loads below.
         const int row_q = sq.start + qbase;
         mbar_arrive_expect_tx(bars.q_full(st), 2 * Q_TILE);
 #pragma unroll
@@ -273,7 +303,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                       h, row_q);
         }
       }
+      for (int q = lane; q < BM; q += 32) {
+        const int qpos = qbase + q;
+        const bool qv = qpos < sq.len;
+        s_lse[st * BM + q] =
+            qv ? p.lse[lse_index(p, b, h, sq.start, qpos)] * 1.4426950408889634f : 0.f;
+        s_dlt[st * BM + q] = qv ? p.delta[static_cast<size_t>(h) * p.total + sq.start + qpos] : 0.f;
+      }
       __syncwarp();
+      if (lane == 0) mbar_arrive(bars.q_full(st));
     }
     for (int t = max(0, n_steps - QS); t < n_steps && !*abort; ++t)
       if (!warp_wait(bars.q_empty(t % QS), (t / QS) & 1, p.err, abort, W_QEMPTY)) break;
@@ -342,89 +380,94 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int st = t % QS;
           if (!(ok = mbar_wait(bars.p_ready(), t & 1, p.err, abort, W_PREADY))) break;
           tc_fence_after();
-          // dV += P^T dO  (A: P^T from TMEM; B: dO MN-major)
+          // dV += P^T dO  (A: P^T from TMEM, queries 0-31 in packed columns
+          // 0-15 and 32-63 in columns 32-47; B: dO MN-major)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8,
+            mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8 + (kk >= 2 ? 16 : 0),
                    sdesc_sw128(sbase + OFF_DO + st * Q_TILE + kk * 2048, Q_CHUNK, 1024), ID_DVK,
                    (t > 0 || kk > 0) ? 1u : 0u);
         }
       }
       tc_commit(bars.dkv_done());
     }
-  } else if (warp < 4) {
+  } else if (warp < WARP_DQ0) {
     // ------------------------------------------------- softmax / dS warps ---
-    const int r = threadIdx.x;            // key row in the tile = TMEM lane
+    // Thread = key row r (TMEM lane); warps w and w+4 share a lane quarter and
+    // take query columns [32 hf, 32 hf + 32) of the 64-wide step.
+    const int r = threadIdx.x & (BN - 1);
+    const int hf = threadIdx.x >> 7;
     const int kpos = j * BN + r;          // key position in the sequence
     const bool key_ok = kpos < sq.len;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    float* s_lse = reinterpret_cast<float*>(smem + OFF_LSE);
-    float* s_dlt = reinterpret_cast<float*>(smem + OFF_DLT);
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float* s_lse = reinterpret_cast<const float*>(smem + OFF_LSE);
+    const float* s_dlt = reinterpret_cast<const float*>(smem + OFF_DLT);
     const float c2 = p.scale_log2;
+    // Visible queries of this key row: qpos in [qlo, qhi).
+    const int qlo = p.causal ? kpos : 0;
+    const int qhi = key_ok ? sq.len : 0;
     bool ok = true;
     for (int t = 0; t < n_steps && ok; ++t) {
-      const int h = hk * g + t / n_qt;
-      const int qbase = (i0 + t % n_qt) * BM;   // first query of the tile
+      const int qbase = (i0 + t % n_qt) * BM + 32 * hf;   // first query of this half
       const int st = t % QS;
-      const float* lse_t = s_lse + st * BM;
-      const float* dlt_t = s_dlt + st * BM;
-      (void)h;
+      const float* lse_t = s_lse + st * BM + 32 * hf;
+      const float* dlt_t = s_dlt + st * BM + 32 * hf;
       // The stage's LSE / D_i values (and Q, dO) have landed.
       if (!(ok = warp_wait(bars.q_full(st), (t / QS) & 1, p.err, abort, W_QFULL))) break;
-      // Visible queries of this key row: qpos in [qlo, qhi).
-      const int qlo = p.causal ? kpos : 0;
-      const int qhi = key_ok ? sq.len : 0;
-
       if (!(ok = warp_wait(bars.s_full(), t & 1, p.err, abort, W_SFULL))) break;
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tmem + lane_off + TM_S, sr[0]);
-      tmem_ld32(tmem + lane_off + TM_S + 32, sr[1]);
+      uint32_t sr[32];
+      tmem_ld32(tmem + lane_off + TM_S + 32 * hf, sr);
       tmem_ld_wait();
-      reg_fence(sr[0]);
-      reg_fence(sr[1]);
-      float pr[BM];
-      uint32_t pk[32];
+      reg_fence(sr);
+      // Whole half visible (no causal edge, no sequence end inside it)?
+      const bool full = qbase >= qlo && qbase + 32 <= qhi;
+      float pr[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int q = 0; q < BM; q += 2) {
-        const int qp = qbase + q;
-        const float s0 = __uint_as_float(sr[q >> 5][q & 31]);
-        const float s1 = __uint_as_float(sr[q >> 5][(q + 1) & 31]);
-        const float p0 = (qp >= qlo && qp < qhi) ? ex2_approx(fmaf(s0, c2, -lse_t[q])) : 0.f;
-        const float p1 = (qp + 1 >= qlo && qp + 1 < qhi) ? ex2_approx(fmaf(s1, c2, -lse_t[q + 1]))
-                                                        : 0.f;
+      for (int q = 0; q < 32; q += 2) {
+        float p0 = ex2_approx(fmaf(__uint_as_float(sr[q]), c2, -lse_t[q]));
+        float p1 = ex2_approx(fmaf(__uint_as_float(sr[q + 1]), c2, -lse_t[q + 1]));
+        if (!full) {
+          const int qp = qbase + q;
+          p0 = (qp >= qlo && qp < qhi) ? p0 : 0.f;
+          p1 = (qp + 1 >= qlo && qp + 1 < qhi) ? p1 : 0.f;
+        }
         pr[q] = p0;
         pr[q + 1] = p1;
         pk[q >> 1] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(tmem + lane_off + TM_S, pk);   // P^T (bf16) over S^T
+      // P^T (bf16, 16 packed columns) over the first half of this half's own
+      // S^T columns, which only this thread has read.
+      tmem_st16(tmem + lane_off + TM_S + 32 * hf, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bars.p_ready());
 
       if (!(ok = warp_wait(bars.dp_full(), t & 1, p.err, abort, W_DPFULL))) break;
       tc_fence_after();
-      uint32_t dr[2][32];
-      tmem_ld32(tmem + lane_off + TM_DP, dr[0]);
-      tmem_ld32(tmem + lane_off + TM_DP + 32, dr[1]);
+      uint32_t dr[32];
+      tmem_ld32(tmem + lane_off + TM_DP + 32 * hf, dr);
       tmem_ld_wait();
-      reg_fence(dr[0]);
-      reg_fence(dr[1]);
-      // dS^T row into the shared buffer t&1 once the MMAs of step t-2 are done.
+      reg_fence(dr);
+      // dS^T row half into the shared buffer t&1 once the MMAs of step t-2
+      // are done with it.
       if (!(ok = warp_wait(bars.ds_empty(t & 1), ((t >> 1) & 1) ^ 1, p.err, abort, W_DSEMPTY)))
         break;
       uint8_t* ds_row = smem + OFF_DS + (t & 1) * DS_TILE + r * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {   // 16-byte chunk c holds queries 8c..8c+7
+      for (int c = 0; c < 4; ++c) {   // 16-byte chunk 4hf+c holds queries 8c..8c+7 of the half
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int q = 8 * c + 2 * e;
-          const float d0 = pr[q] * (__uint_as_float(dr[q >> 5][q & 31]) - dlt_t[q]);
-          const float d1 = pr[q + 1] * (__uint_as_float(dr[q >> 5][(q + 1) & 31]) - dlt_t[q + 1]);
+          const float d0 = pr[q] * (__uint_as_float(dr[q]) - dlt_t[q]);
+          const float d1 = pr[q + 1] * (__uint_as_float(dr[q + 1]) - dlt_t[q + 1]);
           w[e] = pack_bf16x2(d0, d1);
         }
-        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        const int chunk = 4 * hf + c;
+        *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_async_smem();
       tc_fence_before();
@@ -438,7 +481,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + off;
       __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + off;
 #pragma unroll
-      for (int c = 0; c < DP / 32; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * hf + cc;   // 32-column block of the head dim
         uint32_t a[32], v[32];
         tmem_ld32(tmem + lane_off + TM_DK + 32 * c, a);
         tmem_ld32(tmem + lane_off + TM_DV + 32 * c, v);
@@ -464,10 +508,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < WARP_TMA) {
     // ------------------------------------------------------ dQ drain warps ---
-    const int d = (warp - 4) * 32 + lane;     // head-dim row of dQ^T = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    // Thread = head-dim row d of dQ^T (TMEM lane). Each step's 64 x D tile is
+    // written to shared memory as fp32 [query][d] and added into the global
+    // accumulator by one TMA bulk reduce issued by thread d = 0.
+    const int d = (warp - WARP_DQ0) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp - WARP_DQ0) * 32) << 16;
+    float* stage = reinterpret_cast<float*>(smem + OFF_DQS);
     for (int u = 0; u < n_steps; ++u) {
       if (!warp_wait(bars.dq_full(u & 1), (u >> 1) & 1, p.err, abort, W_DQFULL)) break;
       tc_fence_after();
@@ -479,17 +527,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       reg_fence(qr[1]);
       tc_fence_before();
       mbar_arrive(bars.dq_empty(u & 1));
-      const int h = hk * g + u / n_qt;
-      const int qbase = (i0 + u % n_qt) * BM;
+      // The previous step's reduce has finished reading the staging tile.
+      if (!warp_wait(bars.dq_sfree(), (u & 1) ^ 1, p.err, abort, W_DQSFREE)) break;
       if (d < p.D) {
-        const int qn = min(BM, sq.len - qbase);
-        float* dst = p.dq_accum + (static_cast<size_t>(sq.start + qbase) * p.H + h) * p.D + d;
-        const size_t stride = static_cast<size_t>(p.H) * p.D;
 #pragma unroll
-        for (int q = 0; q < BM; ++q)
-          if (q < qn) red_add_f32(dst + q * stride, __uint_as_float(qr[q >> 5][q & 31]));
+        for (int q = 0; q < BM; ++q) stage[q * p.D + d] = __uint_as_float(qr[q >> 5][q & 31]);
+      }
+      fence_async_smem();
+      mbar_arrive(bars.dq_staged());
+      if (d == 0) {
+        // Never leaves the loop on its own (its warp-mates would wait for it
+        // in the next warp_wait); after a failed wait it only skips the add.
+        if (mbar_wait(bars.dq_staged(), u & 1, p.err, abort, W_DQSTAGED)) {
+          const int h = hk * g + u / n_qt;
+          const int row_q = sq.start + (i0 + u % n_qt) * BM;
+          // Rows past the sequence end hold zeros (their dS was masked to 0).
+          tma_reduce_add_3d(&tm_dq, smem_u32(stage), 0, h, row_q);
+          bulk_wait_read();
+        }
+        mbar_arrive(bars.dq_sfree());
       }
     }
+    if (d == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -520,16 +579,17 @@ cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned m
   const long long tiles = static_cast<long long>(num_j) * p.H_kv * p.B;
   if (tiles > INT_MAX) return cudaErrorInvalidConfiguration;
   if (tiles > 0) {
-    CUtensorMap tq, tk, tv, tg;
+    CUtensorMap tq, tk, tv, tg, tdq;
     if (!make_tmap_bf16_3d(&tq, p.q, p.total, p.H, p.D, BM) ||
         !make_tmap_bf16_3d(&tk, p.k, p.total, p.H_kv, p.D, BN) ||
         !make_tmap_bf16_3d(&tv, p.v, p.total, p.H_kv, p.D, BN) ||
-        !make_tmap_bf16_3d(&tg, p.dout, p.total, p.H, p.D, BM))
+        !make_tmap_bf16_3d(&tg, p.dout, p.total, p.H, p.D, BM) ||
+        !make_tmap_f32_3d(&tdq, p.dq_accum, p.total, p.H, p.D, BM))
       return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
-    bwd_main_kernel<<<static_cast<unsigned>(tiles), THREADS, SMEM, stream>>>(tq, tk, tv, tg, p,
-                                                                           num_j);
+    bwd_main_kernel<<<static_cast<unsigned>(tiles), THREADS, SMEM, stream>>>(tq, tk, tv, tg, tdq,
+                                                                           p, num_j);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -54,7 +54,7 @@ enum : unsigned {
 
 template <int D>
 struct FwdCfg {
-  static constexpr int STAGES = (D == 64) ? 4 : 2;
+  static constexpr int STAGES = (D == 64) ? 4 : 3;
   static constexpr int CHUNKS = D / 64;
   static constexpr uint32_t TILE = BM * D * 2;  // bytes of one 128-row tile
   static constexpr uint32_t OFF_Q = 0;

@@ -86,4 +86,9 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long ro
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
                        unsigned box_rows);
 
+// Host: 3-D fp32 view (D, heads, rows) with a (D, 1, box_rows) box and no
+// swizzle, for bulk reduce-adds of [box_rows][D] shared-memory tiles.
+bool make_tmap_f32_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
+                      unsigned box_rows);
+
 }  // namespace fa
