@@ -321,6 +321,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t ID_SDP = idesc_bf16(BN, BM, false, false);   // S^T, dP^T
       constexpr uint32_t ID_DVK = idesc_bf16(BN, DP, false, true);    // dV, dK
       constexpr uint32_t ID_DQ = idesc_bf16(DP, BM, true, true);      // dQ^T
+      // Shared-memory descriptors, built once and stepped by constant offsets.
+      const uint64_t k_kmaj = sdesc_sw128(sbase + OFF_K, 16, 1024);         // K as A (S^T)
+      const uint64_t v_kmaj = sdesc_sw128(sbase + OFF_V, 16, 1024);         // V as A (dP^T)
+      const uint64_t k_mnmaj = sdesc_sw128(sbase + OFF_K, KV_CHUNK, 1024);  // K^T as A (dQ^T)
+      const uint64_t q_kmaj = sdesc_sw128(sbase + OFF_Q, 16, 1024);         // Q as B (S^T)
+      const uint64_t g_kmaj = sdesc_sw128(sbase + OFF_DO, 16, 1024);        // dO as B (dP^T)
+      const uint64_t q_mnmaj = sdesc_sw128(sbase + OFF_Q, Q_CHUNK, 1024);   // Q as B (dK)
+      const uint64_t g_mnmaj = sdesc_sw128(sbase + OFF_DO, Q_CHUNK, 1024);  // dO as B (dV)
+      const uint64_t ds_kmaj = sdesc_sw128(sbase + OFF_DS, 16, 1024);       // dS^T as A (dK)
+      const uint64_t ds_mnmaj = sdesc_sw128(sbase + OFF_DS, KV_CHUNK, 1024);  // dS^T as B (dQ^T)
       bool ok = mbar_wait(bars.kv_full(), 0, p.err, abort, W_KV);
       for (int t = 0; ok && t <= n_steps; ++t) {
         if (t < n_steps) {
@@ -332,8 +342,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int kk = 0; kk < DP / 16; ++kk) {
             const uint32_t ko = (kk >> 2) * KV_CHUNK + (kk & 3) * 32;
             const uint32_t qo = (kk >> 2) * Q_CHUNK + (kk & 3) * 32;
-            mma_ss(tmem + TM_S, sdesc_sw128(sbase + OFF_K + ko, 16, 1024),
-                   sdesc_sw128(sbase + OFF_Q + st * Q_TILE + qo, 16, 1024), ID_SDP, kk > 0);
+            mma_ss(tmem + TM_S, sdesc_add(k_kmaj, ko), sdesc_add(q_kmaj, st * Q_TILE + qo), ID_SDP,
+                   kk > 0);
           }
           tc_commit(bars.s_full());
           // dP^T = V dO^T, once the softmax warps are done with dP^T of t-1.
@@ -344,15 +354,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int kk = 0; kk < DP / 16; ++kk) {
             const uint32_t vo = (kk >> 2) * KV_CHUNK + (kk & 3) * 32;
             const uint32_t go = (kk >> 2) * Q_CHUNK + (kk & 3) * 32;
-            mma_ss(tmem + TM_DP, sdesc_sw128(sbase + OFF_V + vo, 16, 1024),
-                   sdesc_sw128(sbase + OFF_DO + st * Q_TILE + go, 16, 1024), ID_SDP, kk > 0);
+            mma_ss(tmem + TM_DP, sdesc_add(v_kmaj, vo), sdesc_add(g_kmaj, st * Q_TILE + go), ID_SDP,
+                   kk > 0);
           }
           tc_commit(bars.dp_full());
         }
         if (t >= 1) {
           const int u = t - 1;
           const int su = u % QS;
-          const uint32_t ds = sbase + OFF_DS + (u & 1) * DS_TILE;
+          const uint32_t ds_off = (u & 1) * DS_TILE;
           if (t == n_steps &&
               !(ok = mbar_wait(bars.ds_ready(), u & 1, p.err, abort, W_DSREADY)))
             break;
@@ -360,8 +370,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           // dK += dS^T Q   (A: dS^T K-major in smem; B: Q MN-major)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ss(tmem + TM_DK, sdesc_sw128(ds + kk * 32, 16, 1024),
-                   sdesc_sw128(sbase + OFF_Q + su * Q_TILE + kk * 2048, Q_CHUNK, 1024), ID_DVK,
+            mma_ss(tmem + TM_DK, sdesc_add(ds_kmaj, ds_off + kk * 32),
+                   sdesc_add(q_mnmaj, su * Q_TILE + kk * 2048), ID_DVK,
                    (u > 0 || kk > 0) ? 1u : 0u);
           // dQ^T = K^T dS^T  (A: K MN-major; B: dS^T MN-major), into dQ buffer u&1
           if (!(ok = mbar_wait(bars.dq_empty(u & 1), ((u >> 1) & 1) ^ 1, p.err, abort,
@@ -370,8 +380,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ss(tmem + TM_DQ + (u & 1) * BM, sdesc_sw128(sbase + OFF_K + kk * 2048, KV_CHUNK, 1024),
-                   sdesc_sw128(ds + kk * 2048, KV_CHUNK, 1024), ID_DQ, kk > 0);
+            mma_ss(tmem + TM_DQ + (u & 1) * BM, sdesc_add(k_mnmaj, kk * 2048),
+                   sdesc_add(ds_mnmaj, ds_off + kk * 2048), ID_DQ, kk > 0);
           tc_commit(bars.dq_full(u & 1));
           tc_commit(bars.ds_empty(u & 1));
           tc_commit(bars.q_empty(su));
@@ -385,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
             mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8 + (kk >= 2 ? 16 : 0),
-                   sdesc_sw128(sbase + OFF_DO + st * Q_TILE + kk * 2048, Q_CHUNK, 1024), ID_DVK,
+                   sdesc_add(g_mnmaj, st * Q_TILE + kk * 2048), ID_DVK,
                    (t > 0 || kk > 0) ? 1u : 0u);
         }
       }

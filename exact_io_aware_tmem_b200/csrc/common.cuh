@@ -172,6 +172,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The same descriptor with its start address moved by ``bytes`` (a multiple
+// of 16 that keeps the address inside shared memory), so MMA loops can build
+// each descriptor once and step it with one add.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane
 // (warp%4)*32 + t of TMEM. The registers are only valid after tmem_ld_wait().
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {

@@ -17,15 +17,20 @@
 //               separate multi-stage shared-memory rings (mbarrier full/empty
 //               pairs, 128-byte swizzle, no multicast);
 //   warp 5      MMA issuer (one thread): S_j = Q K_j^T with tcgen05.mma into
-//               one of two TMEM score buffers, then O += P_{j-1} V_{j-1} with
+//               one of two TMEM score buffers (Q is the A operand, held in
+//               TMEM, so each tile streams only K and V through shared memory
+//               and the tensor core is not held back by shared-memory
+//               bandwidth), then O += P_{j-1} V_{j-1} with
 //               P read straight from TMEM (it overwrites the first half of its
 //               score buffer as packed bf16); issuing QK_j before PV_{j-1}
 //               lets the softmax of tile j overlap the PV of tile j-1;
-//   warps 0-3   softmax, one thread per query row (TMEM lane = row): loads
+//   warps 0-3   softmax, one thread per query row (TMEM lane = row): first
+//               copies its Q row from the swizzled shared tile into TMEM; then
+//               per tile loads
 //               its 128 scores with tcgen05.ld, masks, takes the row max,
 //               exponentiates, sums, stores P back to TMEM, rescales its O row
 //               in TMEM when the max moved, and finally writes O / l and LSE.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D).
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D), Q [384, 384+D/2).
 #include <limits.h>
 #include <math.h>
 
@@ -43,13 +48,18 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S0 = 0;
 constexpr uint32_t TM_S1 = 128;
 constexpr uint32_t TM_O = 256;
+constexpr uint32_t TM_Q = 384;  // Q tile as packed bf16 (D/2 columns), A operand of Q K^T
 constexpr uint32_t CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16 (one swizzle span)
+// The O accumulator is rescaled only when a row max grows by more than this
+// many powers of two; P entries are then at most 2^8 before the bf16 cast.
+constexpr float RESCALE_LOG2 = 8.f;
 constexpr unsigned FULL = 0xffffffffu;
 
 // Codes recorded in the device error word when a wait gives up.
 enum : unsigned {
   W_Q = 0x10100, W_KEMPTY = 0x10200, W_VEMPTY = 0x10300, W_KFULL = 0x10400,
-  W_VFULL = 0x10500, W_PREADY = 0x10600, W_SFULL = 0x10700, W_ODONE = 0x10800
+  W_VFULL = 0x10500, W_PREADY = 0x10600, W_SFULL = 0x10700, W_ODONE = 0x10800,
+  W_QTMEM = 0x10900
 };
 
 template <int D>
@@ -61,8 +71,9 @@ struct FwdCfg {
   static constexpr uint32_t OFF_K = OFF_Q + TILE;
   static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
   static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
-  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_done
-  static constexpr int NBAR = 1 + 4 * STAGES + 5;
+  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_done,
+  // q_tmem
+  static constexpr int NBAR = 1 + 4 * STAGES + 6;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -79,6 +90,7 @@ struct Bars {
   __device__ uint32_t s_full(int b) const { return base + 8u * (1 + 4 * stages + b); }
   __device__ uint32_t p_ready(int b) const { return base + 8u * (3 + 4 * stages + b); }
   __device__ uint32_t o_done() const { return base + 8u * (5 + 4 * stages); }
+  __device__ uint32_t q_tmem() const { return base + 8u * (6 + 4 * stages); }
 };
 
 // All 32 lanes wait; the warp proceeds only if every lane saw the phase.
@@ -131,6 +143,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bars.p_ready(i), 128);
     }
     mbar_init(bars.o_done(), 1);
+    mbar_init(bars.q_tmem(), 128);
     fence_mbar_init();
   }
   if (warp == WARP_MMA) {
@@ -184,7 +197,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------------------------------ MMA issuer ---
       constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
-      if (mbar_wait(bars.q(), 0, p.err, abort, W_Q)) {
+      // Shared-memory descriptors, built once and stepped by constant offsets.
+      const uint64_t k_desc = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+      const uint64_t v_desc = sdesc_sw128(sbase + C::OFF_V, CHUNK_BYTES, 1024);
+      // Q reaches TMEM through the softmax threads.
+      if (mbar_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM)) {
         tc_fence_after();
         for (int j = 0; j <= n_kv; ++j) {
           if (j < n_kv) {
@@ -196,8 +213,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-              mma_ss(d_s, sdesc_sw128(sbase + C::OFF_Q + off, 16, 1024),
-                     sdesc_sw128(sbase + C::OFF_K + st * C::TILE + off, 16, 1024), IDESC_QK,
+              mma_ts(d_s, tmem + TM_Q + kk * 8, sdesc_add(k_desc, st * C::TILE + off), IDESC_QK,
                      kk > 0);
             }
             tc_commit(bars.s_full(j & 1));
@@ -214,7 +230,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk) {
               mma_ts(tmem + TM_O, a_p + kk * 8,
-                     sdesc_sw128(sbase + C::OFF_V + st * C::TILE + kk * 2048, CHUNK_BYTES, 1024),
+                     sdesc_add(v_desc, st * C::TILE + kk * 2048),
                      IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(bars.v_empty(st));
@@ -232,7 +248,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float c2 = p.scale_log2;
     float m_run = -INFINITY;  // running max of scaled logits, log2 units
     float l_run = 0.f;
-    bool ok = true;
+    // Copy this row of Q from the swizzled shared tile into TMEM as packed
+    // bf16 (even element in the low half): the A operand of S = Q K^T.
+    bool ok = warp_wait(bars.q(), 0, p.err, abort, W_Q);
+    if (ok) {
+#pragma unroll
+      for (int c = 0; c < C::CHUNKS; ++c) {
+        const uint8_t* rowp = smem + C::OFF_Q + c * CHUNK_BYTES + row * 128;
+        uint32_t w[32];
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16) {
+          const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((k16 ^ (row & 7)) << 4));
+          w[4 * k16 + 0] = v.x;
+          w[4 * k16 + 1] = v.y;
+          w[4 * k16 + 2] = v.z;
+          w[4 * k16 + 3] = v.w;
+        }
+        tmem_st32(tmem + lane_off + TM_Q + 32 * c, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bars.q_tmem());
+    }
     for (int j = 0; j < n_kv && ok; ++j) {
       const uint32_t s_col = (j & 1) ? TM_S1 : TM_S0;
       if (!warp_wait(bars.s_full(j & 1), (j >> 1) & 1, p.err, abort, W_SFULL)) {
@@ -255,15 +292,25 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= nvalid) r[c][i] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // Row max with 8 independent partial maxima (no 128-long dependency chain).
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[c][i]));
-      const float m_new = fmaxf(m_run, mx * c2);
+        for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(r[c][i]));
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // The reference max only moves when the row max grows by more than
+      // RESCALE_LOG2 (log2 units): P = 2^(s c - m_ref) then stays below
+      // 2^RESCALE_LOG2, and O / l is the same for any consistent reference.
+      const float m_cand = mx * c2;
+      const bool grow = m_cand > m_run + RESCALE_LOG2;   // always true on the first tile
+      const float m_new = grow ? m_cand : m_run;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2_approx(m_run - m_use);
-      float sum = 0.f;
+      const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -271,9 +318,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 32; i += 2) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2, -m_use));
           const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use));
-          sum += p0 + p1;
+          sum8[(i >> 1) & 7] += p0 + p1;
           pk[c >> 1][(c & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
         }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
+                        ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       // P overwrites the first 64 columns of this score buffer.
       tmem_st32(tmem + lane_off + s_col, pk[0]);
       tmem_st32(tmem + lane_off + s_col + 32, pk[1]);

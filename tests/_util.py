@@ -19,6 +19,20 @@ def max_abs(a, b) -> float:
     return float(np.abs(a - b).max())
 
 
+def o_excess_bf16(got, ref, tol: float = 1.5e-2) -> float:
+    """Largest amount by which |got - ref| exceeds the bf16 output bound.
+
+    The bound is tol on the computed value plus the bf16 cast of the output,
+    which moves it by at most half an ulp, 2^-9 |ref|. Returns <= 0 when every
+    element is inside the bound.
+    """
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if got.size == 0:
+        return -tol
+    return float((np.abs(got - ref) - (tol + np.abs(ref) * 2.0 ** -9)).max())
+
+
 def rel_fro(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)

@@ -2,7 +2,9 @@
 
 Tolerances (from the method's target and the arithmetic):
   float32 path: max-abs <= 1e-5 on O and LSE;
-  bf16 path:    max-abs <= 1.5e-2 on O, max-abs <= 1e-3 on LSE.
+  bf16 path:    |O - O_ref| <= 1.5e-2 + 2^-9 |O_ref| (the bound on the
+                computed value plus at most half a bf16 ulp from casting the
+                output to bf16), max-abs <= 1e-3 on LSE.
 Small cases span several 128-row tiles with ragged tails; the full-size
 workloads are checked on sampled rows the oracle computes one by one.
 """
@@ -13,7 +15,8 @@ import torch
 import exact_io_aware_tmem_b200 as fa
 from exact_io_aware_tmem_b200.workloads import WORKLOADS, make_inputs, random_case
 from oracle import attention as oa
-from tests._util import f64, max_abs, oracle_lse_layout, sample_forward, to_api
+from tests._util import (f64, max_abs, o_excess_bf16, oracle_lse_layout, sample_forward,
+                         to_api)
 
 pytestmark = pytest.mark.gpu
 
@@ -43,12 +46,16 @@ def check_full(inp, causal, scale, B, N, o_tol, lse_tol):
                                           scale)
     T = inp.q.shape[0]
     o = f64(o).reshape(T, inp.q.shape[1], -1)
-    err_o = max_abs(o, o_ref)
     err_l = max_abs(f64(lse), oracle_lse_layout(lse_ref, inp, B, N))
     assert np.isfinite(o).all()
-    assert err_o <= o_tol, f"O max-abs {err_o}"
+    if inp.q.dtype == torch.bfloat16:
+        excess = o_excess_bf16(o, o_ref, o_tol)
+        assert excess <= 0, f"O outside the bf16 bound by {excess} (max-abs {max_abs(o, o_ref)})"
+    else:
+        err_o = max_abs(o, o_ref)
+        assert err_o <= o_tol, f"O max-abs {err_o}"
     assert err_l <= lse_tol, f"LSE max-abs {err_l}"
-    return err_o, err_l
+    return err_l
 
 
 # ------------------------------------------------------------ float32 path ---
@@ -152,6 +159,6 @@ def test_bf16_workload_sampled(name):
             got_lse = f64(lse[h, idx])
         else:
             got_lse = f64(lse[b, h, torch.as_tensor(rows, device=o.device)])
-        assert max_abs(got, o_ref) <= O_TOL_BF16
+        assert o_excess_bf16(got, o_ref, O_TOL_BF16) <= 0
         assert max_abs(got_lse, lse_ref) <= LSE_TOL_BF16
     assert torch.isfinite(o).all()
