@@ -2,8 +2,8 @@
 """Attention forward + backward throughput on B200, one JSON line.
 
 A step is one pass of the whole hot path over one batch of the workload:
-fa_fwd (O, LSE) then fa_bwd (preprocess, fused dK/dV/dQ kernel, dQ
-conversion), all through the C ABI of libfa_b200.so. Inputs are seeded
+fa_fwd (O, LSE) then fa_bwd (preprocess D_i, dK/dV kernel, dQ kernel), all
+through the C ABI of libfa_b200.so. Inputs are seeded
 synthetic Gaussians resident in HBM before the timed region starts.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
@@ -88,7 +88,8 @@ def source_sha(*names) -> str:
 
 
 KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
-                  "bwd_main_kernel": ("bwd_bf16.cu", "common.cuh", "params.h")}
+                  "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
+                  "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h")}
 
 
 def recorded_traffic(kernel: str, workload: str):
@@ -344,7 +345,7 @@ def run_ours(args, w) -> None:
     max_ms = reduce_max(elapsed_ms, dev)
     k_ms = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
             for name, (a, b) in {"fwd_bf16_kernel": (0, 1), "bwd_preprocess": (1, 2),
-                                 "bwd_main_kernel": (2, 3), "bwd_dq_convert": (3, 4)}.items()}
+                                 "bwd_dkdv_kernel": (2, 3), "bwd_dq_kernel": (3, 4)}.items()}
     k_ms = {n: reduce_max(t, dev) for n, t in k_ms.items()}
 
     # End to end through the public API with host buffers: pinned H2D of the
@@ -378,11 +379,16 @@ def run_ours(args, w) -> None:
     per_step_fl = fwd_fl + bwd_fl
     value = aggregate(per_step_fl * args.steps, world, [max_ms / 1e3]) / 1e12
     fwd_tf = fwd_fl / (k_ms["fwd_bf16_kernel"] / 1e3) / 1e12
-    bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_main_kernel"] + k_ms["bwd_dq_convert"]
+    bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_dkdv_kernel"] + k_ms["bwd_dq_kernel"]
     bwd_tf = bwd_fl / (bwd_ms / 1e3) / 1e12
-    # Dominant kernel: the one with the larger share of the step.
-    dom = max(("fwd_bf16_kernel", "bwd_main_kernel"), key=lambda n: k_ms[n])
-    dom_fl = fwd_fl if dom == "fwd_bf16_kernel" else bwd_fl
+    # Dominant kernel: the one with the largest share of the step. Algorithmic
+    # FLOPs per launch: the forward's two products (4 N^2 D per head), the
+    # dK/dV kernel's four (S, dP, dV, dK: 8 N^2 D), the dQ kernel's three
+    # (S, dP again and dQ: 6 N^2 D), causal halving each.
+    kernel_fl = {"fwd_bf16_kernel": fwd_fl, "bwd_dkdv_kernel": 2.0 * fwd_fl,
+                 "bwd_dq_kernel": 1.5 * fwd_fl}
+    dom = max(kernel_fl, key=lambda n: k_ms[n])
+    dom_fl = kernel_fl[dom]
     achieved = dom_fl / (k_ms[dom] / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     line = {

@@ -41,6 +41,7 @@ SIGNATURES = {
                                c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                c_int, c_int, c_float, c_void_p, c_int, c_ll, c_void_p]),
     "fa_get_error_string": (ctypes.c_char_p, [c_int]),
+    "fa_last_cuda_error_string": (ctypes.c_char_p, []),
     "fa_check_device_error": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_uint)]),
     "fa_set_wait_budget": (None, [c_ll]),
     "fa_selftest_wait_timeout": (c_int, [c_ll, c_void_p]),
@@ -54,6 +55,8 @@ class FAError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
         msg = lib().fa_get_error_string(status).decode() if _lib is not None else str(status)
+        if status == FA_ERR_CUDA and _lib is not None:
+            msg += f" ({lib().fa_last_cuda_error_string().decode()})"
         super().__init__(f"{what}: {msg}")
 
 

@@ -18,6 +18,15 @@ __device__ unsigned g_err_word[2];
 namespace {
 
 constexpr long long kDefaultBudget = 4000000000LL;  // ~2 s at 1.9 GHz
+
+// Last CUDA error behind an FA_ERR_CUDA on this host thread.
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+fa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FA_OK;
+  g_last_cuda = e;
+  return FA_ERR_CUDA;
+}
 long long g_budget = kDefaultBudget;
 
 constexpr int kMaxDevices = 64;
@@ -129,21 +138,6 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int h
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_f32_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
-                      unsigned box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
-                              static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4,
-                                 static_cast<cuuint64_t>(heads) * D * 4};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(D), 1, box_rows};
-  const cuuint32_t estride[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
-            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 namespace {
 
 __global__ void wait_selftest_kernel(DevErr e) {
@@ -193,14 +187,14 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (p.err.word == nullptr) return FA_ERR_CUDA;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = (dtype == FA_F32) ? fa::launch_fwd_f32(p, s) : fa::launch_fwd_bf16(p, s);
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return fa::cuda_status(e);
 }
 
 size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype) {
   if (total_tokens < 0 || H <= 0 || D <= 0) return 0;
+  if (dtype != FA_BF16 && dtype != FA_F32) return 0;
   const size_t T = static_cast<size_t>(total_tokens);
-  const size_t dq = (dtype == FA_BF16) ? fa::round256(T * H * D * sizeof(float)) : 0;
-  return dq + fa::round256(T * H * sizeof(float)) + 256;
+  return fa::round256(T * H * sizeof(float)) + 256;
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -240,20 +234,14 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t T = static_cast<size_t>(p.total);
-  if (dtype == FA_BF16) {
-    p.dq_accum = reinterpret_cast<float*>(ws);
-    ws += fa::round256(T * H * D * sizeof(float));
-  }
-  p.delta = reinterpret_cast<float*>(ws);
+  p.delta = static_cast<float*>(workspace);
   p.err.word = fa::err_word();
   if (p.err.word == nullptr) return FA_ERR_CUDA;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e =
       (dtype == FA_F32) ? fa::launch_bwd_f32(p, s) : fa::launch_bwd_bf16(p, s, mask);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return fa::cuda_status(e);
 }
 
 const char* fa_get_error_string(fa_status status) {
@@ -291,6 +279,8 @@ fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream) {
              ? FA_OK
              : FA_ERR_CUDA;
 }
+
+const char* fa_last_cuda_error_string(void) { return cudaGetErrorString(fa::g_last_cuda); }
 
 int fa_version(void) { return 100; }
 

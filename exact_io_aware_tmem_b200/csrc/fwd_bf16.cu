@@ -104,17 +104,19 @@ template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m) {
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m,
+                    int group) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
 
-  // Tile order: the longest causal tiles (largest m_blk) first.
-  const int HB = p.H * p.B;
-  const int m_blk = num_m - 1 - static_cast<int>(blockIdx.x / HB);
-  const int rem = static_cast<int>(blockIdx.x % HB);
+  // Tile order: groups of heads for L2 reuse of K / V; inside a group the
+  // longest causal tiles (largest m_blk) first.
+  const TileSlot ts = grouped_slot(blockIdx.x, num_m, p.H * p.B, group);
+  const int m_blk = num_m - 1 - ts.t;
+  const int rem = ts.unit;
   const int h = rem % p.H;
   const int b = rem / p.H;
   const SeqInfo sq = seq_info(p, b);
@@ -410,8 +412,9 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
+  const int group = l2_group(4ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
   fwd_bf16_kernel<D><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(tq, tk, tv, p,
-                                                                                 num_m);
+                                                                                 num_m, group);
   return cudaGetLastError();
 }
 

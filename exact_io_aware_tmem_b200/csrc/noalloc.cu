@@ -5,9 +5,9 @@
 // not call cudaMalloc - for example a kernel plugin inside a host framework
 // that owns every device allocation, or a latency-critical path where an
 // allocation would synchronise the device or fail under a fixed memory
-// budget. fa_bwd needs a caller-provided workspace (the fp32 dQ accumulator
-// and the D_i row terms); this entry point supplies it from a fixed,
-// file-scope device array instead, and allocates nothing.
+// budget. fa_bwd needs a caller-provided workspace (the D_i row terms); this
+// entry point supplies it from a fixed, file-scope device array instead, and
+// allocates nothing.
 //
 // The array is part of the loaded library: every GPU that loads the library
 // holds FA_NOALLOC_SCRATCH_BYTES of device memory for it until the process
@@ -21,8 +21,8 @@ namespace fa {
 namespace {
 
 // The shared scratch. Its contents persist from call to call; the backward
-// pass re-initialises everything it reads (the preprocess kernel zeroes the
-// dQ accumulator and writes every D_i it uses) before using it.
+// pass re-initialises everything it reads (the preprocess kernel writes every
+// D_i the later kernels use) before using it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;

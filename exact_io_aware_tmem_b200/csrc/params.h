@@ -20,8 +20,7 @@ struct AttnParams {
   void* dq;
   void* dk;
   void* dv;
-  float* dq_accum;  // fp32 [T, H, D] (bf16 backward)
-  float* delta;     // fp32 [H, T]: D_i = dO_i . O_i
+  float* delta;     // fp32 [H, T]: D_i = dO_i . O_i (backward workspace)
   const int* cu_seqlens;  // null for dense batches
   int B, H, H_kv, N, D;
   int causal;
@@ -66,11 +65,40 @@ __device__ __forceinline__ size_t lse_index(const AttnParams& p, int b, int h, i
   return (static_cast<size_t>(b) * p.H + h) * p.N + pos;
 }
 
+// Tile order for L2 reuse. The (sequence, head) units are taken in groups of
+// ``group`` consecutive units, and every tile of a group is launched before
+// the next group's, tile index slowest inside a group: the CTAs running at any
+// time then stream the tensors of a few units only, which stay in L2.
+// Returns the tile index within its unit and the unit.
+struct TileSlot {
+  int t;
+  int unit;
+};
+
+__device__ __forceinline__ TileSlot grouped_slot(unsigned bid, int num_t, int units, int group) {
+  const long long per = static_cast<long long>(num_t) * group;
+  const int gi = static_cast<int>(bid / per);
+  const int gs = min(group, units - gi * group);
+  const int local = static_cast<int>(bid - gi * per);
+  return {local / gs, gi * group + local % gs};
+}
+
+// Host: group size for units that each stream ``bytes_per_unit`` bytes, so that
+// a group's streams fit in about 48 MB of the 126 MB L2; ``share`` consecutive
+// units stream the same tensors (query heads of one key/value head).
+inline int l2_group(long long bytes_per_unit, int share, int units) {
+  const long long budget = 48ll << 20;
+  long long g = (bytes_per_unit > 0 ? budget / bytes_per_unit : units);
+  if (g < 1) g = 1;
+  g *= share;
+  return static_cast<int>(g < units ? g : units);
+}
+
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream);
-// mask: bit 0 preprocess, bit 1 main kernel, bit 2 dQ conversion.
+// mask: bit 0 preprocess (D_i), bit 1 dK/dV kernel, bit 2 dQ kernel.
 cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned mask);
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
 
@@ -85,10 +113,5 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long ro
 // x >= D lie outside the tensor and arrive as zeros.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
                        unsigned box_rows);
-
-// Host: 3-D fp32 view (D, heads, rows) with a (D, 1, box_rows) box and no
-// swizzle, for bulk reduce-adds of [box_rows][D] shared-memory tiles.
-bool make_tmap_f32_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
-                      unsigned box_rows);
 
 }  // namespace fa

@@ -106,10 +106,10 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  fa_stream_t stream);
 
 /*
- * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs for T tokens,
- * H query heads and head dimension D: the float32 dQ accumulator [T, H, D]
- * (bf16 only) and the float32 row terms D_i = dO_i . O_i [H, T], each
- * rounded up to 256 bytes. Returns 0 for invalid sizes.
+ * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs for T tokens
+ * and H query heads: the float32 row terms D_i = dO_i . O_i [H, T], rounded
+ * up to 256 bytes, plus 256. D is checked but does not change the size.
+ * Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype);
 
@@ -142,12 +142,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 
 /*
  * fa_bwd_phases - fa_bwd restricted to some of its three kernels, so that
- * each can be timed by itself: bit 0 = preprocess (D_i = dO_i . O_i and
- * zeroing of the fp32 dQ accumulator), bit 1 = the main tensor-core kernel
- * (recomputation, dK, dV and accumulation of dQ), bit 2 = conversion of the
- * accumulator to dQ. fa_bwd(...) is fa_bwd_phases(7, ...). Phases must be
- * enqueued in that order on the same workspace. For FA_F32 only mask 7 is
- * accepted (FA_ERR_UNSUPPORTED otherwise). Other arguments as for fa_bwd.
+ * each can be timed by itself: bit 0 = preprocess (D_i = dO_i . O_i into the
+ * workspace), bit 1 = the dK / dV kernel, bit 2 = the dQ kernel (bits 1 and 2
+ * both read D_i, so bit 0 must have run on the same workspace first).
+ * fa_bwd(...) is fa_bwd_phases(7, ...). For FA_F32 only mask 7 is accepted
+ * (FA_ERR_UNSUPPORTED otherwise). Other arguments as for fa_bwd.
  */
 fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void* v,
                         const void* o, const float* lse, const void* dout, void* dq, void* dk,
@@ -169,9 +168,8 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
  *
  * Arguments, layouts and results are those of fa_bwd without workspace and
  * ws_bytes. Limit: fa_bwd_workspace_size(T, H, D, dtype) must not exceed
- * FA_NOALLOC_SCRATCH_BYTES (for bf16 about T * H * (D + 1) * 4 bytes, e.g.
- * T * H <= 64000 at D = 128); larger problems return FA_ERR_UNSUPPORTED
- * before anything is enqueued.
+ * FA_NOALLOC_SCRATCH_BYTES (about T * H * 4 bytes, so T * H <= 8,388,000);
+ * larger problems return FA_ERR_UNSUPPORTED before anything is enqueued.
  *
  * The scratch is shared by every call on a device and keeps the last call's
  * contents; each call re-initialises what it reads. Calls whose kernels can
@@ -190,6 +188,13 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
 
 /* fa_get_error_string - static, human-readable name of a status code. */
 const char* fa_get_error_string(fa_status status);
+
+/*
+ * fa_last_cuda_error_string - the CUDA runtime's description of the most
+ * recent CUDA error behind an FA_ERR_CUDA returned on the calling host
+ * thread ("no error" if there was none). Static storage; do not free.
+ */
+const char* fa_last_cuda_error_string(void);
 
 /*
  * fa_check_device_error - synchronises ``stream``, then reports and clears

@@ -45,7 +45,7 @@ def test_version_and_error_strings(lib):
 def test_workspace_size(lib):
     T, H, D = 1000, 16, 128
     r = lambda x: (x + 255) // 256 * 256
-    assert lib.fa_bwd_workspace_size(T, H, D, _abi.FA_BF16) == r(T * H * D * 4) + r(T * H * 4) + 256
+    assert lib.fa_bwd_workspace_size(T, H, D, _abi.FA_BF16) == r(T * H * 4) + 256
     assert lib.fa_bwd_workspace_size(T, H, D, _abi.FA_F32) == r(T * H * 4) + 256
     assert lib.fa_bwd_workspace_size(-1, H, D, _abi.FA_BF16) == 0
 

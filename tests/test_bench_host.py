@@ -74,16 +74,16 @@ def test_peaks_fallback(monkeypatch, tmp_path):
 
 def test_recorded_traffic_needs_matching_source(monkeypatch, tmp_path):
     (tmp_path / "profiles").mkdir()
-    rec = {"bwd_main_kernel": {"workload": "w", "source_sha": "stale", "bytes_per_launch": 5}}
+    rec = {"bwd_dkdv_kernel": {"workload": "w", "source_sha": "stale", "bytes_per_launch": 5}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     real_root = bench.ROOT
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "source_sha", lambda *n: "fresh")
-    assert bench.recorded_traffic("bwd_main_kernel", "w") is None
-    rec["bwd_main_kernel"]["source_sha"] = "fresh"
+    assert bench.recorded_traffic("bwd_dkdv_kernel", "w") is None
+    rec["bwd_dkdv_kernel"]["source_sha"] = "fresh"
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
-    assert bench.recorded_traffic("bwd_main_kernel", "w") == 5
-    assert bench.recorded_traffic("bwd_main_kernel", "other") is None
+    assert bench.recorded_traffic("bwd_dkdv_kernel", "w") == 5
+    assert bench.recorded_traffic("bwd_dkdv_kernel", "other") is None
     assert real_root
 
 

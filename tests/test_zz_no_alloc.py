@@ -120,9 +120,9 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row(lib):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
-    # T * H * (D + 1) * 4 bytes > 32 MiB: refused before anything is enqueued
-    # (no pointer is touched, so none is needed).
-    T, H, D = 70000, 1, 128
+    # T * H * 4 bytes > 32 MiB: refused before anything is enqueued (no pointer
+    # is touched, so none is needed).
+    T, H, D = 9_000_000, 1, 128
     need = lib.fa_bwd_workspace_size(T, H, D, _abi.FA_BF16)
     assert need > SCRATCH_BYTES
     st = lib.fa_bwd_noalloc(None, None, None, None, None, None, None, None, None, 1, H, H, T, D,
