@@ -267,8 +267,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int t = max(0, n_steps - QS); t < n_steps && !*abort; ++t)
       if (!warp_wait(bars.q_empty(t % QS), (t / QS) & 1, p.err, abort, W_QEMPTY)) break;
   } else if (warp == WARP_MMA) {
-    if (lane == 0) {
+    {
       // -------------------------------------------------------- MMA issuer ---
+      // The whole warp runs the loop (waits and operands stay warp-uniform);
+      // one elected lane issues the tensor-core instructions and commits.
+      const uint32_t leader = elect_one();
       constexpr uint32_t ID_SDP = idesc_bf16(BT, BT, false, false);  // S^T, dP^T
       constexpr uint32_t ID_DVK = idesc_bf16(BT, DP, false, true);   // dV, dK
       const uint64_t k_kmaj = sdesc_sw128(sbase + OFF_K, 16, 1024);
@@ -282,23 +285,23 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const uint32_t o = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + TM_S, sdesc_add(k_kmaj, o), sdesc_add(q_kmaj, st * TILE + o), ID_SDP,
+          mma_ss_if(leader, tmem + TM_S, sdesc_add(k_kmaj, o), sdesc_add(q_kmaj, st * TILE + o), ID_SDP,
                  kk > 0);
         }
-        tc_commit(bars.s_full());
+        tc_commit_if(leader, bars.s_full());
       };
       auto issue_dp = [&](int st) {
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const uint32_t o = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + TM_DP, sdesc_add(v_kmaj, o), sdesc_add(g_kmaj, st * TILE + o), ID_SDP,
+          mma_ss_if(leader, tmem + TM_DP, sdesc_add(v_kmaj, o), sdesc_add(g_kmaj, st * TILE + o), ID_SDP,
                  kk > 0);
         }
-        tc_commit(bars.dp_full());
+        tc_commit_if(leader, bars.dp_full());
       };
-      bool ok = mbar_wait(bars.kv_full(), 0, p.err, abort, W_KV);
+      bool ok = warp_wait(bars.kv_full(), 0, p.err, abort, W_KV);
       if (ok && n_steps > 0) {
-        ok = mbar_wait(bars.q_full(0), 0, p.err, abort, W_QFULL);
+        ok = warp_wait(bars.q_full(0), 0, p.err, abort, W_QFULL);
         if (ok) {
           tc_fence_after();
           issue_s(0);
@@ -311,30 +314,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       // dP_{t+1}, and the dS phase of step t overlaps dV_t and S_{t+1}.
       for (int t = 0; ok && t < n_steps; ++t) {
         const int st = t % QS;
-        if (!(ok = mbar_wait(bars.p_ready(), t & 1, p.err, abort, W_PREADY))) break;
+        if (!(ok = warp_wait(bars.p_ready(), t & 1, p.err, abort, W_PREADY))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          mma_ts(tmem + TM_DV, tmem + TM_S + packed_col(kk),
+          mma_ts_if(leader, tmem + TM_DV, tmem + TM_S + packed_col(kk),
                  sdesc_add(g_mn, st * TILE + kk * 2048), ID_DVK, (t > 0 || kk > 0) ? 1u : 0u);
         const bool more = t + 1 < n_steps;
         const int sn = (t + 1) % QS;
         if (more) {
-          if (!(ok = mbar_wait(bars.q_full(sn), ((t + 1) / QS) & 1, p.err, abort, W_QFULL)))
+          if (!(ok = warp_wait(bars.q_full(sn), ((t + 1) / QS) & 1, p.err, abort, W_QFULL)))
             break;
           tc_fence_after();
           issue_s(sn);
         }
-        if (!(ok = mbar_wait(bars.ds_ready(), t & 1, p.err, abort, W_DSREADY))) break;
+        if (!(ok = warp_wait(bars.ds_ready(), t & 1, p.err, abort, W_DSREADY))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          mma_ts(tmem + TM_DK, tmem + TM_DP + packed_col(kk),
+          mma_ts_if(leader, tmem + TM_DK, tmem + TM_DP + packed_col(kk),
                  sdesc_add(q_mn, st * TILE + kk * 2048), ID_DVK, (t > 0 || kk > 0) ? 1u : 0u);
         if (more) issue_dp(sn);
-        tc_commit(bars.q_empty(st));
+        tc_commit_if(leader, bars.q_empty(st));
       }
-      tc_commit(bars.dkv_done());
+      tc_commit_if(leader, bars.dkv_done());
     }
   } else {
     // ------------------------------------------------- softmax / dS warps ---
@@ -559,15 +562,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive_expect_tx(bars.q_full(), 2 * TILE);
       load_tile(sbase + OFF_Q, &tm_q, bars.q_full(), h, row_q);
       load_tile(sbase + OFF_DO, &tm_do, bars.q_full(), h, row_q);
-      for (int jj = 0; jj < n_kv; ++jj) {
-        const int sk = jj % KS, sv = jj % VS;
-        const int row_kv = sq.start + jj * BT;
-        if (!mbar_wait(bars.k_empty(sk), ((jj / KS) & 1) ^ 1, p.err, abort, W_KEMPTY)) break;
-        mbar_arrive_expect_tx(bars.k_full(sk), TILE);
-        load_tile(sbase + OFF_K + sk * TILE, &tm_k, bars.k_full(sk), hk, row_kv);
-        if (!mbar_wait(bars.v_empty(sv), ((jj / VS) & 1) ^ 1, p.err, abort, W_VEMPTY)) break;
-        mbar_arrive_expect_tx(bars.v_full(sv), TILE);
-        load_tile(sbase + OFF_V + sv * TILE, &tm_v, bars.v_full(sv), hk, row_kv);
+      // K and V run through rings of different depth and are loaded
+      // independently (K first when both have a free slot), so a K load
+      // never waits behind a V slot.
+      int jk = 0, jv = 0;
+      long long t_last = clock64();
+      while (jk < n_kv || jv < n_kv) {
+        bool progress = false;
+        if (jk < n_kv && mbar_try_wait(bars.k_empty(jk % KS), ((jk / KS) & 1) ^ 1)) {
+          mbar_arrive_expect_tx(bars.k_full(jk % KS), TILE);
+          load_tile(sbase + OFF_K + (jk % KS) * TILE, &tm_k, bars.k_full(jk % KS), hk,
+                    sq.start + jk * BT);
+          ++jk;
+          progress = true;
+        }
+        if (jv < n_kv && jv < jk && mbar_try_wait(bars.v_empty(jv % VS), ((jv / VS) & 1) ^ 1)) {
+          mbar_arrive_expect_tx(bars.v_full(jv % VS), TILE);
+          load_tile(sbase + OFF_V + (jv % VS) * TILE, &tm_v, bars.v_full(jv % VS), hk,
+                    sq.start + jv * BT);
+          ++jv;
+          progress = true;
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (*abort) {
+          break;
+        } else if (clock64() - t_last > p.err.budget) {
+          *abort = 1;
+          atomicOr(p.err.word, ERR_TIMEOUT);
+          atomicExch(p.err.word + 1, jk < n_kv ? W_KEMPTY : W_VEMPTY);
+          break;
+        }
       }
       // Drain: the tensor core's last arrivals on the empty barriers land
       // before exit.
@@ -577,8 +602,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(bars.v_empty(jj % VS), (jj / VS) & 1, p.err, abort, W_VEMPTY)) break;
     }
   } else if (warp == WARP_MMA) {
-    if (lane == 0) {
+    {
       // -------------------------------------------------------- MMA issuer ---
+      // The whole warp runs the loop (waits and operands stay warp-uniform);
+      // one elected lane issues the tensor-core instructions and commits.
+      const uint32_t leader = elect_one();
       constexpr uint32_t ID_SDP = idesc_bf16(BT, BT, false, false);  // S, dP
       constexpr uint32_t ID_DQ = idesc_bf16(BT, DP, false, true);    // dQ += dS K
       const uint64_t q_kmaj = sdesc_sw128(sbase + OFF_Q, 16, 1024);
@@ -591,25 +619,25 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const uint32_t o = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + TM_S, sdesc_add(q_kmaj, o), sdesc_add(k_kmaj, st * TILE + o), ID_SDP,
+          mma_ss_if(leader, tmem + TM_S, sdesc_add(q_kmaj, o), sdesc_add(k_kmaj, st * TILE + o), ID_SDP,
                  kk > 0);
         }
-        tc_commit(bars.s_full(jj & 1));
+        tc_commit_if(leader, bars.s_full(jj & 1));
       };
       auto issue_dp = [&](int jj) {  // dP_jj = dO V_jj^T; V_jj is free afterwards
         const int st = jj % VS;
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const uint32_t o = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + TM_DP + (jj & 1) * BT, sdesc_add(g_kmaj, o),
+          mma_ss_if(leader, tmem + TM_DP + (jj & 1) * BT, sdesc_add(g_kmaj, o),
                  sdesc_add(v_kmaj, st * TILE + o), ID_SDP, kk > 0);
         }
-        tc_commit(bars.dp_full(jj & 1));
-        tc_commit(bars.v_empty(st));
+        tc_commit_if(leader, bars.dp_full(jj & 1));
+        tc_commit_if(leader, bars.v_empty(st));
       };
-      bool ok = mbar_wait(bars.q_full(), 0, p.err, abort, W_Q) &&
-                mbar_wait(bars.k_full(0), 0, p.err, abort, W_KFULL) &&
-                mbar_wait(bars.v_full(0), 0, p.err, abort, W_VFULL);
+      bool ok = warp_wait(bars.q_full(), 0, p.err, abort, W_Q) &&
+                warp_wait(bars.k_full(0), 0, p.err, abort, W_KFULL) &&
+                warp_wait(bars.v_full(0), 0, p.err, abort, W_VFULL);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -623,28 +651,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int jj = 0; ok && jj < n_kv; ++jj) {
         const int st = jj % KS;
         if (jj + 1 < n_kv) {
-          if (!(ok = mbar_wait(bars.k_full((jj + 1) % KS), ((jj + 1) / KS) & 1, p.err, abort,
+          if (!(ok = warp_wait(bars.k_full((jj + 1) % KS), ((jj + 1) / KS) & 1, p.err, abort,
                                W_KFULL)))
             break;
-          if (!(ok = mbar_wait(bars.s_free(), jj & 1, p.err, abort, W_SFREE))) break;
+          if (!(ok = warp_wait(bars.s_free(), jj & 1, p.err, abort, W_SFREE))) break;
           tc_fence_after();
           issue_s(jj + 1);
-          if (!(ok = mbar_wait(bars.v_full((jj + 1) % VS), ((jj + 1) / VS) & 1, p.err, abort,
+          if (!(ok = warp_wait(bars.v_full((jj + 1) % VS), ((jj + 1) / VS) & 1, p.err, abort,
                                W_VFULL)))
             break;
           tc_fence_after();
           issue_dp(jj + 1);
         }
-        if (!(ok = mbar_wait(bars.ds_ready(jj & 1), (jj >> 1) & 1, p.err, abort, W_DSREADY)))
+        if (!(ok = warp_wait(bars.ds_ready(jj & 1), (jj >> 1) & 1, p.err, abort, W_DSREADY)))
           break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          mma_ts(tmem + TM_DQ, tmem + TM_DP + (jj & 1) * BT + kk * 8,
+          mma_ts_if(leader, tmem + TM_DQ, tmem + TM_DP + (jj & 1) * BT + kk * 8,
                  sdesc_add(k_mn, st * TILE + kk * 2048), ID_DQ, (jj > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bars.k_empty(st));
+        tc_commit_if(leader, bars.k_empty(st));
       }
-      tc_commit(bars.dq_done());
+      tc_commit_if(leader, bars.dq_done());
     }
   } else {
     // ------------------------------------------------- softmax / dS warps ---

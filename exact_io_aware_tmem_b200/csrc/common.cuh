@@ -148,6 +148,52 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// 1 in exactly one lane of a converged warp (the leader elect.sync picks), 0
+// in the others. A warp that issues tensor-core work computes its operands
+// in all lanes and lets the leader issue: the operands then stay warp-uniform.
+__device__ __forceinline__ uint32_t elect_one() {
+  uint32_t leader;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 l;\n\t"
+      "elect.sync l|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(leader));
+  return leader;
+}
+
+// mma_ss / mma_ts / tc_commit issued only where ``leader`` is non-zero.
+__device__ __forceinline__ void mma_ss_if(uint32_t leader, uint32_t d_tmem, uint64_t a_desc,
+                                          uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_if(uint32_t leader, uint32_t d_tmem, uint32_t a_tmem,
+                                          uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_if(uint32_t leader, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %1, 0;\n\t"
+      "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar),
+      "r"(leader)
+      : "memory");
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
 //   15 A major (0 = K, 1 = MN), 16 B major, 17-22 N>>3, 24-28 M>>4.
@@ -239,6 +285,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe instead of the special-function unit, which sustains
+// only 16 exponentials per clock per SM; running a share of a tile's
+// exponentials here lets both pipes work at once. Method: Cody-Waite range
+// reduction x = j + f with j = round(x) and |f| <= 1/2 (the rounding is done
+// by adding 1.5 * 2^23, which leaves j in the low mantissa bits), 2^f from a
+// degree-3 polynomial fitted for least maximum relative error on [-1/2, 1/2]
+// (linear-programming fit; bound 7.5e-5, well under bf16's 2^-9 rounding of
+// P), and 2^j applied by adding j to the exponent field. Valid for
+// x <= 127; inputs below -125 (masked scores are -inf) are clamped to -125, so
+// the result is then about 2^-125 rather than 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  x = fmaxf(x, -125.f);
+  const float t = x + kRound;
+  const float j = t - kRound;
+  const float f = x - j;
+  const float p =
+      fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); ``lo`` in bits 0-15.

@@ -12,25 +12,35 @@
 // in base 2 on pre-scaled logits (scale * log2 e), which is the same
 // recurrence up to rounding.
 //
-// How, on B200 (one CTA per 128-row Q tile, 192 threads):
-//   warp 4      TMA producer: Q tile once, then K_j and V_j tiles through
+// How, on B200 (one CTA per 128-row Q tile, 320 threads):
+//   warp 8      TMA producer: Q tile once, then K_j and V_j tiles through
 //               separate multi-stage shared-memory rings (mbarrier full/empty
 //               pairs, 128-byte swizzle, no multicast);
-//   warp 5      MMA issuer (one thread): S_j = Q K_j^T with tcgen05.mma into
-//               one of two TMEM score buffers (Q is the A operand, held in
-//               TMEM, so each tile streams only K and V through shared memory
-//               and the tensor core is not held back by shared-memory
-//               bandwidth), then O += P_{j-1} V_{j-1} with
-//               P read straight from TMEM (it overwrites the first half of its
-//               score buffer as packed bf16); issuing QK_j before PV_{j-1}
-//               lets the softmax of tile j overlap the PV of tile j-1;
-//   warps 0-3   softmax, one thread per query row (TMEM lane = row): first
-//               copies its Q row from the swizzled shared tile into TMEM; then
-//               per tile loads
-//               its 128 scores with tcgen05.ld, masks, takes the row max,
-//               exponentiates, sums, stores P back to TMEM, rescales its O row
-//               in TMEM when the max moved, and finally writes O / l and LSE.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D), Q [384, 384+D/2).
+//   warp 9      MMA issuer (one thread): S_j = Q K_j^T with tcgen05.mma into
+//               TMEM score buffer j mod 2 (Q is the A operand, held in TMEM,
+//               so each tile streams only K and V through shared memory and
+//               the tensor core is not held back by shared-memory bandwidth),
+//               and O += P_j V_j with P read straight from its own TMEM
+//               columns as packed bf16. S_{j+2} is issued as soon as the
+//               softmax has loaded S_j, ahead of PV_j;
+//   warps 0-7   softmax, two groups of four warps; group g takes the key
+//               tiles j = g, g+2, g+4, ... One thread per query row (TMEM
+//               lane = row): it loads its 128 scores with tcgen05.ld,
+//               releases the score buffer, masks, takes the row max,
+//               exponentiates, sums, stores P to TMEM and rescales its O row
+//               in TMEM when the reference max moved. Group 0 first copies Q
+//               from the swizzled shared tile into TMEM. At the end both
+//               groups merge their row sums and each writes half of O / l.
+// The two groups run the same recurrence with one shared reference max per
+// row: the group on tile j takes the reference of tile j-1 from the other
+// group (a shared-memory word per row, published by an mbarrier arrive as
+// soon as that tile's row max is known, long before its exponentials are
+// done), so the exponential work of neighbouring tiles overlaps instead of
+// running back to back. Each group keeps its own partial row sum l_g, in the
+// reference of its own last tile; O has a single accumulator whose reference
+// is always the latest one, which is what lets P_j V_j add into it directly.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D), Q [384, 384+D/2),
+// P [448, 512).
 #include <limits.h>
 #include <math.h>
 
@@ -41,25 +51,32 @@ namespace {
 
 constexpr int BM = 128;  // query rows per CTA (= TMEM lanes)
 constexpr int BN = 128;  // keys per tile
-constexpr int WARP_TMA = 4;
-constexpr int WARP_MMA = 5;
-constexpr int THREADS = 192;
+constexpr int WARP_TMA = 8;
+constexpr int WARP_MMA = 9;
+constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S0 = 0;
-constexpr uint32_t TM_S1 = 128;
 constexpr uint32_t TM_O = 256;
 constexpr uint32_t TM_Q = 384;  // Q tile as packed bf16 (D/2 columns), A operand of Q K^T
+constexpr uint32_t TM_P = 448;  // P tile as packed bf16 (64 columns), A operand of P V
 constexpr uint32_t CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16 (one swizzle span)
-// The O accumulator is rescaled only when a row max grows by more than this
+// The reference max only moves when a row max exceeds it by more than this
 // many powers of two; P entries are then at most 2^8 before the bf16 cast.
 constexpr float RESCALE_LOG2 = 8.f;
 constexpr unsigned FULL = 0xffffffffu;
+// Of every 16 score pairs in a 32-column chunk, this many take their
+// exponentials on the FMA pipe (exp2_poly) and the rest on the
+// special-function unit.
+#ifndef FA_FWD_POLY_PAIRS
+#define FA_FWD_POLY_PAIRS 0
+#endif
+constexpr int POLY_PAIRS = FA_FWD_POLY_PAIRS;
 
 // Codes recorded in the device error word when a wait gives up.
 enum : unsigned {
   W_Q = 0x10100, W_KEMPTY = 0x10200, W_VEMPTY = 0x10300, W_KFULL = 0x10400,
-  W_VFULL = 0x10500, W_PREADY = 0x10600, W_SFULL = 0x10700, W_ODONE = 0x10800,
-  W_QTMEM = 0x10900
+  W_VFULL = 0x10500, W_PREADY = 0x10600, W_SFULL = 0x10700, W_PVDONE = 0x10800,
+  W_QTMEM = 0x10900, W_SFREE = 0x10A00, W_MREF = 0x10B00, W_FIN = 0x10C00
 };
 
 template <int D>
@@ -71,11 +88,16 @@ struct FwdCfg {
   static constexpr uint32_t OFF_K = OFF_Q + TILE;
   static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
   static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
-  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_done,
-  // q_tmem
-  static constexpr int NBAR = 1 + 4 * STAGES + 6;
+  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
+  // mref[2], pv_done[2], p_ready, q_tmem, fin
+  static constexpr int NBAR = 1 + 4 * STAGES + 11;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+  // Once Q is in TMEM its shared tile holds the per-row exchange words:
+  // reference max per group [2][128], then final (m, l) per group [2][2][128].
+  static constexpr uint32_t OFF_MREF = OFF_Q;
+  static constexpr uint32_t OFF_FIN = OFF_Q + 2 * BM * 4;
+  static_assert(OFF_FIN + 4 * BM * 4 <= TILE, "exchange words fit in the Q tile");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -88,9 +110,12 @@ struct Bars {
   __device__ uint32_t v_full(int s) const { return base + 8u * (1 + 2 * stages + s); }
   __device__ uint32_t v_empty(int s) const { return base + 8u * (1 + 3 * stages + s); }
   __device__ uint32_t s_full(int b) const { return base + 8u * (1 + 4 * stages + b); }
-  __device__ uint32_t p_ready(int b) const { return base + 8u * (3 + 4 * stages + b); }
-  __device__ uint32_t o_done() const { return base + 8u * (5 + 4 * stages); }
-  __device__ uint32_t q_tmem() const { return base + 8u * (6 + 4 * stages); }
+  __device__ uint32_t s_free(int b) const { return base + 8u * (3 + 4 * stages + b); }
+  __device__ uint32_t mref(int g) const { return base + 8u * (5 + 4 * stages + g); }
+  __device__ uint32_t pv_done(int g) const { return base + 8u * (7 + 4 * stages + g); }
+  __device__ uint32_t p_ready() const { return base + 8u * (9 + 4 * stages); }
+  __device__ uint32_t q_tmem() const { return base + 8u * (10 + 4 * stages); }
+  __device__ uint32_t fin() const { return base + 8u * (11 + 4 * stages); }
 };
 
 // All 32 lanes wait; the warp proceeds only if every lane saw the phase.
@@ -142,10 +167,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
-      mbar_init(bars.p_ready(i), 128);
+      mbar_init(bars.s_free(i), 128);
+      mbar_init(bars.mref(i), 128);
+      mbar_init(bars.pv_done(i), 1);
     }
-    mbar_init(bars.o_done(), 1);
+    mbar_init(bars.p_ready(), 128);
     mbar_init(bars.q_tmem(), 128);
+    mbar_init(bars.fin(), 256);
     fence_mbar_init();
   }
   if (warp == WARP_MMA) {
@@ -168,22 +196,46 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int c = 0; c < C::CHUNKS; ++c)
         tma_load_2d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), h * D + c * 64, row_q);
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        const int row_kv = sq.start + j * BN;
-        if (!mbar_wait(bars.k_empty(st), ph ^ 1, p.err, abort, W_KEMPTY)) break;
-        mbar_arrive_expect_tx(bars.k_full(st), C::TILE);
+      // K and V run through separate rings and are loaded independently, K
+      // first whenever both have a free slot: K_j is consumed early (QK_j
+      // runs two tiles ahead of PV_j), and a K load that waited behind a V
+      // slot would stall the score MMAs on the slowest event of the loop.
+      int jk = 0, jv = 0;
+      long long t_last = clock64();
+      while (jk < n_kv || jv < n_kv) {
+        bool progress = false;
+        if (jk < n_kv && mbar_try_wait(bars.k_empty(jk % C::STAGES),
+                                       ((jk / C::STAGES) & 1) ^ 1)) {
+          const int st = jk % C::STAGES;
+          mbar_arrive_expect_tx(bars.k_full(st), C::TILE);
 #pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_2d(sbase + C::OFF_K + st * C::TILE + c * CHUNK_BYTES, &tm_k, bars.k_full(st),
-                      hk * D + c * 64, row_kv);
-        if (!mbar_wait(bars.v_empty(st), ph ^ 1, p.err, abort, W_VEMPTY)) break;
-        mbar_arrive_expect_tx(bars.v_full(st), C::TILE);
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_2d(sbase + C::OFF_K + st * C::TILE + c * CHUNK_BYTES, &tm_k,
+                        bars.k_full(st), hk * D + c * 64, sq.start + jk * BN);
+          ++jk;
+          progress = true;
+        }
+        if (jv < n_kv && jv < jk &&
+            mbar_try_wait(bars.v_empty(jv % C::STAGES), ((jv / C::STAGES) & 1) ^ 1)) {
+          const int st = jv % C::STAGES;
+          mbar_arrive_expect_tx(bars.v_full(st), C::TILE);
 #pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_2d(sbase + C::OFF_V + st * C::TILE + c * CHUNK_BYTES, &tm_v, bars.v_full(st),
-                      hk * D + c * 64, row_kv);
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_2d(sbase + C::OFF_V + st * C::TILE + c * CHUNK_BYTES, &tm_v,
+                        bars.v_full(st), hk * D + c * 64, sq.start + jv * BN);
+          ++jv;
+          progress = true;
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (*abort) {
+          break;
+        } else if (clock64() - t_last > p.err.budget) {
+          *abort = 1;
+          atomicOr(p.err.word, ERR_TIMEOUT);
+          atomicExch(p.err.word + 1, jk < n_kv ? W_KEMPTY : W_VEMPTY);
+          break;
+        }
       }
       // Drain: the tensor core's arrivals on the last stages' empty barriers
       // must land before the CTA's shared memory is released.
@@ -195,86 +247,103 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == WARP_MMA) {
-    if (lane == 0) {
-      // ------------------------------------------------------ MMA issuer ---
-      constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
-      constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
-      // Shared-memory descriptors, built once and stepped by constant offsets.
-      const uint64_t k_desc = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
-      const uint64_t v_desc = sdesc_sw128(sbase + C::OFF_V, CHUNK_BYTES, 1024);
-      // Q reaches TMEM through the softmax threads.
-      if (mbar_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM)) {
-        tc_fence_after();
-        for (int j = 0; j <= n_kv; ++j) {
-          if (j < n_kv) {
-            // S_j = Q K_j^T: M=128, N=128, K=D in steps of 16.
-            const int st = j % C::STAGES;
-            if (!mbar_wait(bars.k_full(st), (j / C::STAGES) & 1, p.err, abort, W_KFULL)) break;
-            tc_fence_after();
-            const uint32_t d_s = tmem + ((j & 1) ? TM_S1 : TM_S0);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-              mma_ts(d_s, tmem + TM_Q + kk * 8, sdesc_add(k_desc, st * C::TILE + off), IDESC_QK,
-                     kk > 0);
-            }
-            tc_commit(bars.s_full(j & 1));
-            tc_commit(bars.k_empty(st));
-          }
-          if (j >= 1) {
-            // O += P_t V_t for t = j - 1: M=128, N=D, K=128 keys in steps of 16.
-            const int t = j - 1;
-            const int st = t % C::STAGES;
-            if (!mbar_wait(bars.p_ready(t & 1), (t >> 1) & 1, p.err, abort, W_PREADY)) break;
-            if (!mbar_wait(bars.v_full(st), (t / C::STAGES) & 1, p.err, abort, W_VFULL)) break;
-            tc_fence_after();
-            const uint32_t a_p = tmem + ((t & 1) ? TM_S1 : TM_S0);
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              mma_ts(tmem + TM_O, a_p + kk * 8,
-                     sdesc_add(v_desc, st * C::TILE + kk * 2048),
-                     IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc_commit(bars.v_empty(st));
-            tc_commit(bars.o_done());
-          }
+    // -------------------------------------------------------- MMA issuer ---
+    // The whole warp runs the loop (waits and operands stay warp-uniform);
+    // one elected lane issues the tensor-core instructions and commits.
+    const uint32_t leader = elect_one();
+    constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
+    constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
+    // Shared-memory descriptors, built once and stepped by constant offsets.
+    const uint64_t k_desc = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+    const uint64_t v_desc = sdesc_sw128(sbase + C::OFF_V, CHUNK_BYTES, 1024);
+    // Q reaches TMEM through the softmax threads.
+    bool ok = warp_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM);
+    if (ok) tc_fence_after();
+    // S_j = Q K_j^T into score buffer j mod 2 (M=128, N=128, K=D in steps
+    // of 16) for j = jq; the buffer is free once its group has loaded
+    // S_{j-2}. QK_0 and QK_1 go first, then QK_{j+2} ahead of each PV_j.
+    int jq = 0;
+    for (int j = -2; j < n_kv && ok; ++j) {
+      for (; jq < n_kv && jq <= j + 2; ++jq) {
+        const int st = jq % C::STAGES;
+        if (!warp_wait(bars.k_full(st), (jq / C::STAGES) & 1, p.err, abort, W_KFULL) ||
+            (jq >= 2 &&
+             !warp_wait(bars.s_free(jq & 1), ((jq - 2) >> 1) & 1, p.err, abort, W_SFREE))) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t d_s = tmem + TM_S0 + (jq & 1) * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
+          mma_ts_if(leader, d_s, tmem + TM_Q + kk * 8, sdesc_add(k_desc, st * C::TILE + off),
+                    IDESC_QK, kk > 0);
+        }
+        tc_commit_if(leader, bars.s_full(jq & 1));
+        tc_commit_if(leader, bars.k_empty(st));
       }
+      if (!ok) break;
+      if (j < 0) continue;
+      // O += P_j V_j: M=128, N=D, K=128 keys in steps of 16.
+      const int st = j % C::STAGES;
+      if (!warp_wait(bars.p_ready(), j & 1, p.err, abort, W_PREADY)) break;
+      if (!warp_wait(bars.v_full(st), (j / C::STAGES) & 1, p.err, abort, W_VFULL)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        mma_ts_if(leader, tmem + TM_O, tmem + TM_P + kk * 8,
+                  sdesc_add(v_desc, st * C::TILE + kk * 2048), IDESC_PV,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc_commit_if(leader, bars.v_empty(st));
+      tc_commit_if(leader, bars.pv_done(j & 1));
     }
   } else {
     // ---------------------------------------------------------- softmax ---
-    const int row = threadIdx.x;  // 0..127 = TMEM lane
+    const int g = warp >> 2;            // softmax group: key tiles g, g+2, ...
+    const int quarter = warp & 3;       // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
     const int qpos = m_blk * BM + row;
     const int lim = p.causal ? min(qpos, sq.len - 1) : sq.len - 1;  // last visible key
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float c2 = p.scale_log2;
-    float m_run = -INFINITY;  // running max of scaled logits, log2 units
-    float l_run = 0.f;
-    // Copy this row of Q from the swizzled shared tile into TMEM as packed
-    // bf16 (even element in the low half): the A operand of S = Q K^T.
-    bool ok = warp_wait(bars.q(), 0, p.err, abort, W_Q);
-    if (ok) {
+    float* mref_s = reinterpret_cast<float*>(smem + C::OFF_MREF);
+    float* fin_s = reinterpret_cast<float*>(smem + C::OFF_FIN);
+    float m_g = -INFINITY;  // reference of this group's last tile (log2 units)
+    float l_g = 0.f;        // this group's row sum, in that reference
+    bool ok = true;
+    if (g == 0) {
+      // Copy this row of Q from the swizzled shared tile into TMEM as packed
+      // bf16 (even element in the low half): the A operand of S = Q K^T.
+      ok = warp_wait(bars.q(), 0, p.err, abort, W_Q);
+      if (ok) {
 #pragma unroll
-      for (int c = 0; c < C::CHUNKS; ++c) {
-        const uint8_t* rowp = smem + C::OFF_Q + c * CHUNK_BYTES + row * 128;
-        uint32_t w[32];
+        for (int c = 0; c < C::CHUNKS; ++c) {
+          const uint8_t* rowp = smem + C::OFF_Q + c * CHUNK_BYTES + row * 128;
+          uint32_t w[32];
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16) {
-          const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((k16 ^ (row & 7)) << 4));
-          w[4 * k16 + 0] = v.x;
-          w[4 * k16 + 1] = v.y;
-          w[4 * k16 + 2] = v.z;
-          w[4 * k16 + 3] = v.w;
+          for (int k16 = 0; k16 < 8; ++k16) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((k16 ^ (row & 7)) << 4));
+            w[4 * k16 + 0] = v.x;
+            w[4 * k16 + 1] = v.y;
+            w[4 * k16 + 2] = v.z;
+            w[4 * k16 + 3] = v.w;
+          }
+          tmem_st32(tmem + lane_off + TM_Q + 32 * c, w);
         }
-        tmem_st32(tmem + lane_off + TM_Q + 32 * c, w);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bars.q_tmem());
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bars.q_tmem());
+    } else {
+      // The Q tile's shared memory is reused for the exchange words below:
+      // group 1 writes none before group 0 has finished copying Q out of it.
+      ok = warp_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM);
     }
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const uint32_t s_col = (j & 1) ? TM_S1 : TM_S0;
-      if (!warp_wait(bars.s_full(j & 1), (j >> 1) & 1, p.err, abort, W_SFULL)) {
+    for (int j = g; j < n_kv && ok; j += 2) {
+      const uint32_t s_col = TM_S0 + g * BN;
+      if (!warp_wait(bars.s_full(g), (j >> 1) & 1, p.err, abort, W_SFULL)) {
         ok = false;
         break;
       }
@@ -285,6 +354,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+      // The scores are in registers: the tensor core may overwrite this buffer.
+      tc_fence_before();
+      mbar_arrive(bars.s_free(g));
 
       const int nvalid = lim - j * BN + 1;  // visible keys in this tile
       if (nvalid < BN) {
@@ -304,66 +376,98 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(r[c][i]));
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // The reference max only moves when the row max grows by more than
+      // Reference of tile j-1, published by the other group.
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        if (!warp_wait(bars.mref(g ^ 1), ((j - 1) >> 1) & 1, p.err, abort, W_MREF)) {
+          ok = false;
+          break;
+        }
+        m_prev = mref_s[(g ^ 1) * BM + row];
+      }
+      // The reference only moves when the row max exceeds it by more than
       // RESCALE_LOG2 (log2 units): P = 2^(s c - m_ref) then stays below
       // 2^RESCALE_LOG2, and O / l is the same for any consistent reference.
       const float m_cand = mx * c2;
-      const bool grow = m_cand > m_run + RESCALE_LOG2;   // always true on the first tile
-      const float m_new = grow ? m_cand : m_run;
+      const bool grow = m_cand > m_prev + RESCALE_LOG2;   // always true on tile 0
+      const float m_new = grow ? m_cand : m_prev;
+      mref_s[g * BM + row] = m_new;
+      mbar_arrive(bars.mref(g));
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = grow ? ex2_approx(m_run - m_use) : 1.f;
-      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use));
-          sum8[(i >> 1) & 7] += p0 + p1;
+          const float x0 = fmaf(__uint_as_float(r[c][i]), c2, -m_use);
+          const float x1 = fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use);
+          const bool poly = ((i >> 1) % 16) >= 16 - POLY_PAIRS;   // resolved at compile time
+          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+          sum4[(i >> 1) & 3] += p0 + p1;
           pk[c >> 1][(c & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
         }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
-                        ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-      // P overwrites the first 64 columns of this score buffer.
-      tmem_st32(tmem + lane_off + s_col, pk[0]);
-      tmem_st32(tmem + lane_off + s_col + 32, pk[1]);
-      tmem_st_wait();
-      l_run = l_run * alpha + sum;
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      // This group's partial sum moves to the new reference.
+      l_g = (m_g == m_new) ? l_g + sum : l_g * ex2_approx(m_g - m_use) + sum;
+      m_g = m_new;
       if (j > 0) {
-        // O holds PV_{j-1} once o_done completes; rescale it before PV_j.
-        if (!warp_wait(bars.o_done(), (j - 1) & 1, p.err, abort, W_ODONE)) {
+        // PV_{j-1} (the other group's tile; the tensor core runs PVs in
+        // order) has finished reading P and adding into O once its pv_done
+        // phase completes: P_j may then be stored and O moved to the new
+        // reference before PV_j.
+        if (!warp_wait(bars.pv_done(g ^ 1), ((j - 1) >> 1) & 1, p.err, abort, W_PVDONE)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(FULL, alpha != 1.f)) {
+      }
+      tmem_st32(tmem + lane_off + TM_P, pk[0]);
+      tmem_st32(tmem + lane_off + TM_P + 32, pk[1]);
+      if (j > 0 && __any_sync(FULL, grow)) {
+        const float alpha = grow ? ex2_approx(m_prev - m_use) : 1.f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
-            tmem_ld_wait();
-            reg_fence(o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
+          tmem_ld_wait();
+          reg_fence(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem + lane_off + TM_O + 32 * c, o);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem + lane_off + TM_O + 32 * c, o);
         }
       }
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bars.p_ready(j & 1));
-      m_run = m_new;
+      mbar_arrive(bars.p_ready());
     }
     // ----------------------------------------------------------- epilogue ---
-    if (ok && warp_wait(bars.o_done(), (n_kv - 1) & 1, p.err, abort, W_ODONE)) {
+    // Merge the two partial sums in the final reference (the larger of the
+    // two groups' last references: references never decrease), then each
+    // group writes half of the columns of O / l.
+    if (ok) {
+      fin_s[(2 * g) * BM + row] = m_g;
+      fin_s[(2 * g + 1) * BM + row] = l_g;
+      mbar_arrive(bars.fin());
+      ok = warp_wait(bars.fin(), 0, p.err, abort, W_FIN);
+    }
+    const int last = n_kv - 1;
+    if (ok && warp_wait(bars.pv_done(last & 1), (last >> 1) & 1, p.err, abort, W_PVDONE)) {
       tc_fence_after();
-      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      const float m_o = fin_s[(2 * (g ^ 1)) * BM + row];
+      const float l_o = fin_s[(2 * (g ^ 1) + 1) * BM + row];
+      const float m_fin = fmaxf(m_g, m_o);
+      float l = 0.f;
+      if (m_g != -INFINITY) l += (m_g == m_fin) ? l_g : l_g * ex2_approx(m_g - m_fin);
+      if (m_o != -INFINITY) l += (m_o == m_fin) ? l_o : l_o * ex2_approx(m_o - m_fin);
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       const bool store = qpos < sq.len;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
                             (static_cast<size_t>(sq.start + qpos) * p.H + h) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int c = g * (D / 64) + cc;   // this group's 32-column chunks
         uint32_t o[32];
         tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
         tmem_ld_wait();
@@ -381,9 +485,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (store) {
-        const float lse = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f
-                                        : -INFINITY;
+      if (store && g == 0) {
+        const float lse = (l > 0.f) ? (m_fin + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         p.lse[lse_index(p, b, h, sq.start, qpos)] = lse;
       }
     }
