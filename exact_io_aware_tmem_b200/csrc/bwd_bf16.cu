@@ -285,8 +285,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const uint32_t o = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          mma_ss_if(leader, tmem + TM_S, sdesc_add(k_kmaj, o), sdesc_add(q_kmaj, st * TILE + o), ID_SDP,
-                 kk > 0);
+          mma_ss_if(leader, tmem + TM_S, sdesc_add(k_kmaj, o), sdesc_add(q_kmaj, st * TILE + o),
+                    ID_SDP, kk > 0);
         }
         tc_commit_if(leader, bars.s_full());
       };
@@ -294,8 +294,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk) {
           const uint32_t o = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          mma_ss_if(leader, tmem + TM_DP, sdesc_add(v_kmaj, o), sdesc_add(g_kmaj, st * TILE + o), ID_SDP,
-                 kk > 0);
+          mma_ss_if(leader, tmem + TM_DP, sdesc_add(v_kmaj, o), sdesc_add(g_kmaj, st * TILE + o),
+                    ID_SDP, kk > 0);
         }
         tc_commit_if(leader, bars.dp_full());
       };
@@ -372,10 +372,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool full = qbase >= qlo && qbase + 64 <= qhi;
       float pr[64];
       uint32_t pk[32];
+      // LSE and D_i are read four at a time (one broadcast load per four
+      // columns): per-element loads would crowd the shared-memory pipe the
+      // tensor core's operand reads and the mbarrier polls also use.
+      const float4* lse4 = reinterpret_cast<const float4*>(lse_t);
 #pragma unroll
       for (int q = 0; q < 64; q += 2) {
-        float p0 = ex2_approx(fmaf(__uint_as_float(sr[q >> 5][q & 31]), c2, -lse_t[q]));
-        float p1 = ex2_approx(fmaf(__uint_as_float(sr[q >> 5][(q + 1) & 31]), c2, -lse_t[q + 1]));
+        const float4 l4 = lse4[q >> 2];
+        const float la = (q & 2) ? l4.z : l4.x;
+        const float lb = (q & 2) ? l4.w : l4.y;
+        float p0 = ex2_approx(fmaf(__uint_as_float(sr[q >> 5][q & 31]), c2, -la));
+        float p1 = ex2_approx(fmaf(__uint_as_float(sr[q >> 5][(q + 1) & 31]), c2, -lb));
         if (!full) {
           const int qp = qbase + q;
           p0 = (qp >= qlo && qp < qhi) ? p0 : 0.f;
@@ -400,10 +407,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       reg_fence(dr[0]);
       reg_fence(dr[1]);
       uint32_t dk[32];
+      const float4* dlt4 = reinterpret_cast<const float4*>(dlt_t);
 #pragma unroll
       for (int q = 0; q < 64; q += 2) {
-        const float d0 = pr[q] * (__uint_as_float(dr[q >> 5][q & 31]) - dlt_t[q]);
-        const float d1 = pr[q + 1] * (__uint_as_float(dr[q >> 5][(q + 1) & 31]) - dlt_t[q + 1]);
+        const float4 d4 = dlt4[q >> 2];
+        const float da = (q & 2) ? d4.z : d4.x;
+        const float db = (q & 2) ? d4.w : d4.y;
+        const float d0 = pr[q] * (__uint_as_float(dr[q >> 5][q & 31]) - da);
+        const float d1 = pr[q + 1] * (__uint_as_float(dr[q >> 5][(q + 1) & 31]) - db);
         dk[q >> 1] = pack_bf16x2(d0, d1);
       }
       // dS^T over the first 32 of this half's own 64 dP^T columns.

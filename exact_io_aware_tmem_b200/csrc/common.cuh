@@ -56,6 +56,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete yet may be
+// suspended (up to about 2 microseconds) until it completes, instead of
+// spinning and taking issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(2000)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase of ``bar`` with the given parity has completed. Gives
 // up after ``e.budget`` cycles, or at once when another thread of the CTA has
 // already given up (``*abort`` set): it then records the failure in the
@@ -64,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const D
                                           volatile int* abort, unsigned where) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_suspend(bar, parity)) {
     if (*abort) return false;
     if (clock64() - t0 > e.budget) {
       *abort = 1;
@@ -285,27 +300,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe instead of the special-function unit, which sustains
-// only 16 exponentials per clock per SM; running a share of a tile's
-// exponentials here lets both pipes work at once. Method: Cody-Waite range
-// reduction x = j + f with j = round(x) and |f| <= 1/2 (the rounding is done
-// by adding 1.5 * 2^23, which leaves j in the low mantissa bits), 2^f from a
-// degree-3 polynomial fitted for least maximum relative error on [-1/2, 1/2]
-// (linear-programming fit; bound 7.5e-5, well under bf16's 2^-9 rounding of
-// P), and 2^j applied by adding j to the exponent field. Valid for
-// x <= 127; inputs below -125 (masked scores are -inf) are clamped to -125, so
-// the result is then about 2^-125 rather than 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-  x = fmaxf(x, -125.f);
-  const float t = x + kRound;
-  const float j = t - kRound;
-  const float f = x - j;
-  const float p =
-      fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); ``lo`` in bits 0-15.

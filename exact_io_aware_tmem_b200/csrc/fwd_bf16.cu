@@ -64,13 +64,6 @@ constexpr uint32_t CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16 (one swizzle 
 // many powers of two; P entries are then at most 2^8 before the bf16 cast.
 constexpr float RESCALE_LOG2 = 8.f;
 constexpr unsigned FULL = 0xffffffffu;
-// Of every 16 score pairs in a 32-column chunk, this many take their
-// exponentials on the FMA pipe (exp2_poly) and the rest on the
-// special-function unit.
-#ifndef FA_FWD_POLY_PAIRS
-#define FA_FWD_POLY_PAIRS 0
-#endif
-constexpr int POLY_PAIRS = FA_FWD_POLY_PAIRS;
 
 // Codes recorded in the device error word when a wait gives up.
 enum : unsigned {
@@ -287,8 +280,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (j < 0) continue;
       // O += P_j V_j: M=128, N=D, K=128 keys in steps of 16.
       const int st = j % C::STAGES;
-      if (!warp_wait(bars.p_ready(), j & 1, p.err, abort, W_PREADY)) break;
       if (!warp_wait(bars.v_full(st), (j / C::STAGES) & 1, p.err, abort, W_VFULL)) break;
+      if (!warp_wait(bars.p_ready(), j & 1, p.err, abort, W_PREADY)) break;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk) {
@@ -400,11 +393,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float x0 = fmaf(__uint_as_float(r[c][i]), c2, -m_use);
-          const float x1 = fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use);
-          const bool poly = ((i >> 1) % 16) >= 16 - POLY_PAIRS;   // resolved at compile time
-          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use));
           sum4[(i >> 1) & 3] += p0 + p1;
           pk[c >> 1][(c & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
         }
