@@ -153,3 +153,130 @@ def flops(w_or_lengths, H: int, D: int, causal: bool) -> tuple:
     if causal:
         fwd *= 0.5
     return fwd, 2.5 * fwd
+
+
+# ------------------------------------------------------------------ decode ---
+#
+# Decode inputs: the q_len newest tokens of B sequences against each
+# sequence's key/value cache. The recipe draws, from one
+# ``torch.Generator('cpu').manual_seed(seed)``: Q ``[B*q_len, H, D]``, then the
+# K cache and the V cache ``[rows, H_kv, D]`` as float32 N(0, 1) (cast to the
+# workload dtype), then, for a paged cache, one permutation of all block ids
+# (``torch.randperm``) handed out to the sequences in order. Cache rows that no
+# sequence position uses are set to ``fill`` (NaN by default) so that a kernel
+# which read them would show it.
+
+
+@dataclasses.dataclass
+class DecodeInputs:
+    q: torch.Tensor                    # [B*q_len, H, D]
+    k_cache: torch.Tensor              # [rows, H_kv, D]
+    v_cache: torch.Tensor              # [rows, H_kv, D]
+    cache_seqlens: torch.Tensor        # int32 [B]
+    block_table: Optional[torch.Tensor]  # int32 [B, max_blocks] (paged) or None
+    page_size: int                     # paged: rows per page; contiguous: per-sequence stride
+    q_len: int
+
+    @property
+    def paged(self) -> bool:
+        return self.block_table is not None
+
+
+def decode_case(seed: int, *, dtype: str, lengths: list, q_len: int, H: int, H_kv: int, D: int,
+                page_size: Optional[int] = None, stride: Optional[int] = None,
+                extra_blocks: int = 3, fill: float = float("nan")) -> DecodeInputs:
+    """Seeded decode case; paged when ``page_size`` is given, else contiguous.
+
+    Contiguous: sequence b owns rows [b*stride, b*stride + stride) with
+    ``stride`` (default: the longest length) >= every length. Paged: sequence
+    b owns ceil(len_b / page_size) pages of a shared pool that also holds
+    ``extra_blocks`` unused pages; unused block-table entries are -1.
+    """
+    g = torch.Generator("cpu").manual_seed(seed)
+    B = len(lengths)
+    q = torch.randn((B * q_len, H, D), generator=g)
+    if page_size is None:
+        stride = max(lengths) if stride is None else stride
+        assert stride >= max(lengths)
+        rows = B * stride
+        used = torch.zeros(rows, dtype=torch.bool)
+        for b, n in enumerate(lengths):
+            used[b * stride:b * stride + n] = True
+        table = None
+        ps = stride
+    else:
+        pages = [-(-n // page_size) for n in lengths]
+        n_blocks = sum(pages) + extra_blocks
+        rows = n_blocks * page_size
+        used = torch.zeros(rows, dtype=torch.bool)
+        table = torch.full((B, max(max(pages), 1)), -1, dtype=torch.int32)
+        ps = page_size
+    k = torch.randn((rows, H_kv, D), generator=g)
+    v = torch.randn((rows, H_kv, D), generator=g)
+    if table is not None:
+        perm = torch.randperm(n_blocks, generator=g)
+        nxt = 0
+        for b, n in enumerate(lengths):
+            for i in range(pages[b]):
+                blk = int(perm[nxt])
+                nxt += 1
+                table[b, i] = blk
+                m = min(page_size, n - i * page_size)
+                used[blk * page_size:blk * page_size + m] = True
+    q, k, v = (_to_dtype(x, dtype) for x in (q, k, v))
+    k[~used] = fill
+    v[~used] = fill
+    return DecodeInputs(q, k, v, torch.tensor(lengths, dtype=torch.int32), table, ps, q_len)
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    q_len: int
+    H: int
+    H_kv: int
+    D: int
+    len_lo: int            # cache lengths drawn uniformly from [len_lo, len_hi]
+    len_hi: int
+    page_size: Optional[int]
+    seed: int
+    causal: bool = True
+    dtype: str = "bf16"
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    def lengths(self) -> list:
+        g = torch.Generator("cpu").manual_seed(self.seed + 1000)
+        return torch.randint(self.len_lo, self.len_hi + 1, (self.B,), generator=g).tolist()
+
+
+# Decode workloads (no configuration on the pages or in the task fixes these;
+# they are sized so the caches are far larger than L2): GQA 32/8 heads, D=128,
+# 16 sequences with cache lengths in [4096, 32768]; one new token per sequence,
+# or 8 (a speculative-decoding verify step), over a contiguous or a paged cache.
+DECODE_WORKLOADS = {
+    "bf16_decode_b16_h32_kv8_d128_q1": DecodeWorkload(
+        "bf16_decode_b16_h32_kv8_d128_q1", 16, 1, 32, 8, 128, 4096, 32768, None, 11),
+    "bf16_decode_paged64_b16_h32_kv8_d128_q1": DecodeWorkload(
+        "bf16_decode_paged64_b16_h32_kv8_d128_q1", 16, 1, 32, 8, 128, 4096, 32768, 64, 12),
+    "bf16_decode_b16_h32_kv8_d128_q8": DecodeWorkload(
+        "bf16_decode_b16_h32_kv8_d128_q8", 16, 8, 32, 8, 128, 4096, 32768, None, 13),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload) -> DecodeInputs:
+    return decode_case(w.seed, dtype=w.dtype, lengths=w.lengths(), q_len=w.q_len, H=w.H,
+                       H_kv=w.H_kv, D=w.D, page_size=w.page_size)
+
+
+def decode_bytes(lengths, H_kv: int, D: int, elem: int = 2) -> float:
+    """K and V cache bytes a decode step must read: 2 * sum(len) * H_kv * D * elem."""
+    return 2.0 * sum(int(n) for n in lengths) * H_kv * D * elem
+
+
+def decode_flops(lengths, q_len: int, H: int, D: int) -> float:
+    """4 * q_len * H * D * sum(len): the two products over every cached key."""
+    return 4.0 * q_len * H * D * sum(int(n) for n in lengths)
