@@ -1,9 +1,10 @@
 """Exact IO-aware attention for B200 (sm_100a): tcgen05 / TMEM / TMA kernels.
 
-``fwd`` and ``bwd`` call the C ABI of libfa_b200.so (see include/fa.h).
+``fwd``, ``bwd`` and ``decode`` call the C ABI of libfa_b200.so (see include/fa.h).
 """
-from .attention import (bwd, check_device_error, default_scale, fwd, selftest_wait_timeout,
+from .attention import (bwd, check_device_error, decode, decode_num_splits,
+                        decode_workspace_size, default_scale, fwd, selftest_wait_timeout,
                         set_wait_budget, workspace_size)
 
-__all__ = ["fwd", "bwd", "workspace_size", "check_device_error", "selftest_wait_timeout",
-           "set_wait_budget", "default_scale"]
+__all__ = ["fwd", "bwd", "workspace_size", "decode", "decode_num_splits", "decode_workspace_size",
+           "check_device_error", "selftest_wait_timeout", "set_wait_budget", "default_scale"]

@@ -109,6 +109,50 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return dq, dk, dv
 
 
+def decode_num_splits(B: int, H_kv: int, max_seqlen_k: int, n_split: int = 0) -> int:
+    return int(_abi.lib().fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split))
+
+
+def decode_workspace_size(B: int, q_len: int, H: int, H_kv: int, D: int, max_seqlen_k: int,
+                          n_split: int = 0) -> int:
+    return int(_abi.lib().fa_decode_workspace_size(B, q_len, H, H_kv, D, max_seqlen_k, n_split))
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           cache_seqlens: torch.Tensor, *, q_len: int, max_seqlen_k: int,
+           block_table: Optional[torch.Tensor] = None, page_size: Optional[int] = None,
+           causal: bool = True, scale: Optional[float] = None, n_split: int = 0,
+           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None):
+    """Split-KV decode (fa_decode): O [B*q_len, H, D] bf16 and LSE [B*q_len, H].
+
+    ``q`` is [B*q_len, H, D]; the caches are [rows, H_kv, D]. Contiguous
+    cache: ``page_size`` is the rows per sequence (default: rows // B).
+    Paged cache: ``block_table`` [B, max_blocks] int32 and ``page_size``.
+    """
+    B = cache_seqlens.numel()
+    H, D = q.shape[1], q.shape[2]
+    H_kv = k_cache.shape[1]
+    rows = k_cache.shape[0]
+    if block_table is None and page_size is None:
+        page_size = rows // max(B, 1)
+    max_blocks = block_table.shape[1] if block_table is not None else 0
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[0], H), device=q.device, dtype=torch.float32)
+    need = decode_workspace_size(B, q_len, H, H_kv, D, max_seqlen_k, n_split)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    st = _abi.lib().fa_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), _ptr(cache_seqlens),
+        _ptr(block_table), B, int(q_len), H, H_kv, D, int(page_size), int(max_blocks), rows,
+        int(max_seqlen_k), int(causal), -1.0 if scale is None else float(scale), int(n_split),
+        _ptr(workspace) if need else None, need, _stream(q.device))
+    _abi.check(st, "fa_decode")
+    return out, lse
+
+
 def check_device_error(device: Optional[torch.device] = None) -> tuple:
     """Synchronise the current stream; return (status, where) and clear the flag."""
     import ctypes

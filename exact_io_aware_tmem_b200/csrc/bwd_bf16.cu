@@ -63,15 +63,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
   return __all_sync(FULL, ok);
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
 // One 128-row tile (both 64-column halves of the padded head dim).
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                           int head, int row) {
@@ -798,10 +789,10 @@ cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned m
   if (!(mask & 6u)) return cudaSuccess;
   const int num_t = (p.max_seqlen + BT - 1) / BT;
   CUtensorMap tq, tk, tv, tg;
-  if (!make_tmap_bf16_3d(&tq, p.q, p.total, p.H, p.D, BT) ||
-      !make_tmap_bf16_3d(&tk, p.k, p.total, p.H_kv, p.D, BT) ||
-      !make_tmap_bf16_3d(&tv, p.v, p.total, p.H_kv, p.D, BT) ||
-      !make_tmap_bf16_3d(&tg, p.dout, p.total, p.H, p.D, BT))
+  if (!make_tmap_bf16_3d(&tq, p.q, p.total, p.H, p.D, 1, BT) ||
+      !make_tmap_bf16_3d(&tk, p.k, p.total, p.H_kv, p.D, 1, BT) ||
+      !make_tmap_bf16_3d(&tv, p.v, p.total, p.H_kv, p.D, 1, BT) ||
+      !make_tmap_bf16_3d(&tg, p.dout, p.total, p.H, p.D, 1, BT))
     return cudaErrorInvalidValue;
   if (mask & 2u) {
     const long long tiles = static_cast<long long>(num_t) * p.H_kv * p.B;

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/fa.h"
@@ -124,14 +125,14 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long ro
 }
 
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
-                       unsigned box_rows) {
+                       unsigned box_heads, unsigned box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
                               static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                                  static_cast<cuuint64_t>(heads) * D * 2};
-  const cuuint32_t box[3] = {64, 1, box_rows};
+  const cuuint32_t box[3] = {64, box_heads, box_rows};
   const cuuint32_t estride[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -188,6 +189,107 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = (dtype == FA_F32) ? fa::launch_fwd_f32(p, s) : fa::launch_fwd_bf16(p, s);
   return fa::cuda_status(e);
+}
+
+int fa_decode_num_splits(int B, int H_kv, int max_seqlen_k, int requested) {
+  if (B <= 0 || H_kv <= 0 || max_seqlen_k <= 0) return 1;
+  const long long tiles = (static_cast<long long>(max_seqlen_k) + 127) / 128;
+  long long n = requested;
+  if (n <= 0) {
+    const long long units = static_cast<long long>(B) * H_kv;
+    n = (4 * 148 + units - 1) / units;   // about four CTAs per SM of a 148-SM B200
+  }
+  n = std::max<long long>(1, std::min(n, tiles));
+  const long long chunk = (tiles + n - 1) / n;
+  return static_cast<int>((tiles + chunk - 1) / chunk);
+}
+
+size_t fa_decode_workspace_size(int B, int q_len, int H, int H_kv, int D, int max_seqlen_k,
+                                int n_split) {
+  if (B <= 0 || q_len <= 0 || H <= 0 || H_kv <= 0 || D <= 0 || max_seqlen_k < 0) return 0;
+  const int ns = fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split);
+  if (ns <= 1) return 0;
+  const size_t rows = static_cast<size_t>(ns) * B * q_len * H;
+  return fa::round256(rows * D * 4) + fa::round256(rows * 4);
+}
+
+fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                    const int* cache_seqlens, const int* block_table, int B, int q_len, int H,
+                    int H_kv, int D, int page_size, int max_blocks, long long cache_rows,
+                    int max_seqlen_k, int causal, float scale, int n_split, void* workspace,
+                    size_t ws_bytes, fa_stream_t stream) {
+  if (B < 0 || q_len <= 0 || H <= 0 || H_kv <= 0 || D <= 0 || max_seqlen_k < 0 ||
+      cache_rows < 0 || n_split < 0)
+    return FA_ERR_INVALID_ARG;
+  if (H % H_kv != 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  const int g = H / H_kv;
+  if (static_cast<long long>(q_len) * g > 128) return FA_ERR_UNSUPPORTED;
+  if (cache_rows >= (1ll << 31) || static_cast<long long>(B) * q_len > INT32_MAX ||
+      static_cast<long long>(B) * H_kv > (1ll << 24))
+    return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  if (page_size <= 0 || cache_rows < 1) return FA_ERR_INVALID_ARG;
+  if (block_table == nullptr) {
+    if (page_size < max_seqlen_k) return FA_ERR_INVALID_ARG;
+    if (cache_rows < static_cast<long long>(B - 1) * page_size + max_seqlen_k)
+      return FA_ERR_INVALID_ARG;
+  } else {
+    if (page_size % 16 != 0 || !(128 % page_size == 0 || page_size % 128 == 0))
+      return FA_ERR_UNSUPPORTED;
+    if (max_blocks < (max_seqlen_k + page_size - 1) / page_size || cache_rows % page_size != 0)
+      return FA_ERR_INVALID_ARG;
+  }
+  if (!q || !k_cache || !v_cache || !o || !lse || !cache_seqlens) return FA_ERR_INVALID_ARG;
+  if (!fa::aligned16(q) || !fa::aligned16(k_cache) || !fa::aligned16(v_cache) ||
+      !fa::aligned16(o))
+    return FA_ERR_INVALID_ARG;
+  const int ns = fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split);
+  const size_t need = fa_decode_workspace_size(B, q_len, H, H_kv, D, max_seqlen_k, n_split);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !fa::aligned16(workspace)))
+    return FA_ERR_INVALID_ARG;
+
+  AttnParams p = {};
+  p.q = q;
+  p.k = k_cache;
+  p.v = v_cache;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.D = D;
+  p.N = 0;
+  p.causal = causal;
+  p.max_seqlen = max_seqlen_k;
+  p.total = static_cast<long long>(B) * q_len;
+  if (!(scale > 0.f) || !isfinite(scale)) scale = 1.f / sqrtf(static_cast<float>(D));
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err.budget = fa::g_budget;
+  p.err.word = fa::err_word();
+  if (p.err.word == nullptr) return FA_ERR_CUDA;
+
+  fa::DecodeArgs d = {};
+  d.cache_seqlens = cache_seqlens;
+  d.block_table = block_table;
+  d.page = page_size;
+  d.max_blocks = (block_table != nullptr) ? max_blocks : 0;
+  d.cache_rows = cache_rows;
+  d.q_len = q_len;
+  d.g = g;
+  d.n_rows = q_len * g;
+  d.n_split = ns;
+  const int tiles = std::max(1, (max_seqlen_k + 127) / 128);
+  d.chunk = (tiles + ns - 1) / ns;
+  if (ns > 1) {
+    const size_t rows = static_cast<size_t>(ns) * B * q_len * H;
+    d.o_part = static_cast<float*>(workspace);
+    d.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          fa::round256(rows * D * 4));
+  }
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return fa::cuda_status(fa::launch_decode_bf16(p, d, s));
 }
 
 size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype) {

@@ -69,7 +69,8 @@ constexpr unsigned FULL = 0xffffffffu;
 enum : unsigned {
   W_Q = 0x10100, W_KEMPTY = 0x10200, W_VEMPTY = 0x10300, W_KFULL = 0x10400,
   W_VFULL = 0x10500, W_PREADY = 0x10600, W_SFULL = 0x10700, W_PVDONE = 0x10800,
-  W_QTMEM = 0x10900, W_SFREE = 0x10A00, W_MREF = 0x10B00, W_FIN = 0x10C00
+  W_QTMEM = 0x10900, W_SFREE = 0x10A00, W_MREF = 0x10B00, W_FIN = 0x10C00, W_VFIX = 0x10D00,
+  W_VTAIL = 0x10E00, BAD_CACHE_LEN = 0x10F01, BAD_PAGE = 0x10F02
 };
 
 template <int D>
@@ -82,8 +83,8 @@ struct FwdCfg {
   static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
   static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
   // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
-  // mref[2], pv_done[2], p_ready, q_tmem, fin
-  static constexpr int NBAR = 1 + 4 * STAGES + 11;
+  // mref[2], pv_done[2], p_ready, q_tmem, fin, v_fix
+  static constexpr int NBAR = 1 + 4 * STAGES + 12;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   // Once Q is in TMEM its shared tile holds the per-row exchange words:
@@ -109,7 +110,13 @@ struct Bars {
   __device__ uint32_t p_ready() const { return base + 8u * (9 + 4 * stages); }
   __device__ uint32_t q_tmem() const { return base + 8u * (10 + 4 * stages); }
   __device__ uint32_t fin() const { return base + 8u * (11 + 4 * stages); }
+  __device__ uint32_t v_fix() const { return base + 8u * (12 + 4 * stages); }
 };
+
+__device__ __forceinline__ void record_bounds(const DevErr& e, unsigned where) {
+  atomicOr(e.word, ERR_BOUNDS);
+  atomicExch(e.word + 1, where);
+}
 
 // All 32 lanes wait; the warp proceeds only if every lane saw the phase.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DevErr& e,
@@ -118,30 +125,79 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
   return __all_sync(FULL, ok);
 }
 
-template <int D>
+// DEC = false: the forward over packed or dense sequences (one CTA per 128-row
+// Q tile). DEC = true: split-KV decode, one CTA per (sequence, kv head, key
+// split); its Q tile is the q_len newest tokens x the g query heads of the kv
+// head (rows r = token * g + head), and it writes that split's partial O / l
+// and LSE (or the final O and LSE when there is one split).
+template <int D, bool DEC>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m,
-                    int group) {
+                    int group, const DecodeArgs dec) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
 
-  // Tile order: groups of heads for L2 reuse of K / V; inside a group the
-  // longest causal tiles (largest m_blk) first.
-  const TileSlot ts = grouped_slot(blockIdx.x, num_m, p.H * p.B, group);
-  const int m_blk = num_m - 1 - ts.t;
-  const int rem = ts.unit;
-  const int h = rem % p.H;
-  const int b = rem / p.H;
-  const SeqInfo sq = seq_info(p, b);
-  if (!seq_ok(p, sq) || m_blk * BM >= sq.len) return;  // whole CTA, before any shared state
-  const int hk = h / (p.H / p.H_kv);
-  const int n_kv_all = (sq.len + BN - 1) / BN;
-  const int n_kv = p.causal ? min(n_kv_all, m_blk + 1) : n_kv_all;
+  int m_blk = 0, h = 0, hk = 0, b = 0;
+  int j0 = 0;       // first key tile of this CTA
+  int n_kv = 0;     // key tiles of this CTA
+  int split = 0;
+  SeqInfo sq{0, 0}; // forward: the sequence; decode: start 0, len = keys in cache
+  if constexpr (!DEC) {
+    // Tile order: groups of heads for L2 reuse of K / V; inside a group the
+    // longest causal tiles (largest m_blk) first.
+    const TileSlot ts = grouped_slot(blockIdx.x, num_m, p.H * p.B, group);
+    m_blk = num_m - 1 - ts.t;
+    const int rem = ts.unit;
+    h = rem % p.H;
+    b = rem / p.H;
+    sq = seq_info(p, b);
+    if (!seq_ok(p, sq) || m_blk * BM >= sq.len) return;  // whole CTA, before any shared state
+    hk = h / (p.H / p.H_kv);
+    const int n_kv_all = (sq.len + BN - 1) / BN;
+    n_kv = p.causal ? min(n_kv_all, m_blk + 1) : n_kv_all;
+  } else {
+    split = blockIdx.x % dec.n_split;
+    const int rem = blockIdx.x / dec.n_split;
+    hk = rem % p.H_kv;
+    b = rem / p.H_kv;
+    sq.len = __ldg(dec.cache_seqlens + b);
+    if (sq.len < 0 || sq.len > p.max_seqlen) {
+      if (threadIdx.x == 0) record_bounds(p.err, BAD_CACHE_LEN);
+      return;
+    }
+    j0 = split * dec.chunk;
+    n_kv = min((sq.len + BN - 1) / BN - j0, dec.chunk);
+    if (n_kv <= 0) {
+      // No key in this split: LSE -inf and O 0, so the merge gives it no
+      // weight (the whole output when the sequence is empty).
+      const int r = threadIdx.x;
+      if (r < dec.n_rows) {
+        const int tok = b * dec.q_len + r / dec.g;
+        const int hq = hk * dec.g + r % dec.g;
+        const size_t row = static_cast<size_t>(tok) * p.H + hq;
+        if (dec.n_split == 1) {
+          p.lse[row] = -INFINITY;
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row * D);
+          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+        } else {
+          const size_t prow = static_cast<size_t>(split) * p.total * p.H + row;
+          dec.lse_part[prow] = -INFINITY;
+          float4* dst = reinterpret_cast<float4*>(dec.o_part + prow * D);
+          for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      return;
+    }
+  }
+  // Decode: the split holding the sequence's last, partly filled key tile
+  // zeroes that tile's V rows past the end (the cache may hold anything
+  // there, and 0 * NaN in P V would not be 0) before PV reads it.
+  const bool v_tail = DEC && j0 + n_kv == (sq.len + BN - 1) / BN && (sq.len % BN) != 0;
 
   const Bars bars{sbase + C::OFF_BAR, C::STAGES};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -167,6 +223,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bars.p_ready(), 128);
     mbar_init(bars.q_tmem(), 128);
     mbar_init(bars.fin(), 256);
+    mbar_init(bars.v_fix(), 1);
     fence_mbar_init();
   }
   if (warp == WARP_MMA) {
@@ -179,16 +236,59 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == WARP_TMA) {
+    // ------------------------------------------------------ TMA producer ---
+    // K / V tile jt (absolute key tile) into shared memory at ``dst``.
+    auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int jt) {
+      if constexpr (!DEC) {
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, sq.start + jt * BN);
+      } else if (dec.block_table == nullptr) {
+        const int row = b * dec.page + jt * BN;
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, row);
+      } else {
+        // Paged: one box per page (or one 128-row box inside a larger page).
+        // Pages past the sequence's end load from beyond the cache: zeros.
+        const int box = min(dec.page, BN);
+        for (int u = 0; u < BN / box; ++u) {
+          const int key = jt * BN + u * box;
+          int row = static_cast<int>(dec.cache_rows);
+          if (key < sq.len) {
+            const int pg = key / dec.page;
+            const int blk = (pg < dec.max_blocks)
+                                ? __ldg(dec.block_table + static_cast<size_t>(b) * dec.max_blocks + pg)
+                                : -1;
+            if (blk >= 0 && static_cast<long long>(blk + 1) * dec.page <= dec.cache_rows)
+              row = blk * dec.page + key % dec.page;
+            else
+              record_bounds(p.err, BAD_PAGE);
+          }
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_2d(dst + c * CHUNK_BYTES + u * box * 128, map, bar, hk * D + c * 64, row);
+        }
+      }
+    };
     if (lane == 0) {
-      // ---------------------------------------------------- TMA producer ---
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const int row_q = sq.start + m_blk * BM;
-      mbar_arrive_expect_tx(bars.q(), C::TILE);
+      if constexpr (!DEC) {
+        const int row_q = sq.start + m_blk * BM;
+        mbar_arrive_expect_tx(bars.q(), C::TILE);
 #pragma unroll
-      for (int c = 0; c < C::CHUNKS; ++c)
-        tma_load_2d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), h * D + c * 64, row_q);
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_2d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), h * D + c * 64, row_q);
+      } else {
+        // q_len tokens x g heads: one (64, g, q_len) box per column block.
+        mbar_arrive_expect_tx(bars.q(), dec.n_rows * 128 * C::CHUNKS);
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c)
+          tma_load_3d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), c * 64, hk * dec.g,
+                      b * dec.q_len);
+      }
       // K and V run through separate rings and are loaded independently, K
       // first whenever both have a free slot: K_j is consumed early (QK_j
       // runs two tiles ahead of PV_j), and a K load that waited behind a V
@@ -201,10 +301,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                        ((jk / C::STAGES) & 1) ^ 1)) {
           const int st = jk % C::STAGES;
           mbar_arrive_expect_tx(bars.k_full(st), C::TILE);
-#pragma unroll
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_2d(sbase + C::OFF_K + st * C::TILE + c * CHUNK_BYTES, &tm_k,
-                        bars.k_full(st), hk * D + c * 64, sq.start + jk * BN);
+          load_kv(sbase + C::OFF_K + st * C::TILE, &tm_k, bars.k_full(st), j0 + jk);
           ++jk;
           progress = true;
         }
@@ -212,10 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_try_wait(bars.v_empty(jv % C::STAGES), ((jv / C::STAGES) & 1) ^ 1)) {
           const int st = jv % C::STAGES;
           mbar_arrive_expect_tx(bars.v_full(st), C::TILE);
-#pragma unroll
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_2d(sbase + C::OFF_V + st * C::TILE + c * CHUNK_BYTES, &tm_v,
-                        bars.v_full(st), hk * D + c * 64, sq.start + jv * BN);
+          load_kv(sbase + C::OFF_V + st * C::TILE, &tm_v, bars.v_full(st), j0 + jv);
           ++jv;
           progress = true;
         }
@@ -230,6 +324,27 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
       }
+    }
+    if (v_tail) {
+      // Zero the rows past the sequence's end of the last V tile once it has
+      // landed, then publish them to the tensor core (v_fix).
+      const int t = n_kv - 1;
+      const int st = t % C::STAGES;
+      if (warp_wait(bars.v_full(st), (t / C::STAGES) & 1, p.err, abort, W_VTAIL)) {
+        const int first = sq.len - (j0 + t) * BN;   // rows [first, 128) are past the end
+        uint8_t* tile = smem + C::OFF_V + st * C::TILE;
+        for (int i = lane; i < (BN - first) * 8 * C::CHUNKS; i += 32) {
+          const int c = i / ((BN - first) * 8);
+          const int rr = first + (i / 8) % (BN - first);
+          *reinterpret_cast<uint4*>(tile + c * CHUNK_BYTES + rr * 128 + (i % 8) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.v_fix());
+      }
+    }
+    if (lane == 0) {
       // Drain: the tensor core's arrivals on the last stages' empty barriers
       // must land before the CTA's shared memory is released.
       for (int j = max(0, n_kv - C::STAGES); j < n_kv && !*abort; ++j) {
@@ -281,6 +396,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // O += P_j V_j: M=128, N=D, K=128 keys in steps of 16.
       const int st = j % C::STAGES;
       if (!warp_wait(bars.v_full(st), (j / C::STAGES) & 1, p.err, abort, W_VFULL)) break;
+      if (v_tail && j == n_kv - 1 && !warp_wait(bars.v_fix(), 0, p.err, abort, W_VFIX)) break;
       if (!warp_wait(bars.p_ready(), j & 1, p.err, abort, W_PREADY)) break;
       tc_fence_after();
 #pragma unroll
@@ -297,8 +413,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int g = warp >> 2;            // softmax group: key tiles g, g+2, ...
     const int quarter = warp & 3;       // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const int qpos = m_blk * BM + row;
-    const int lim = p.causal ? min(qpos, sq.len - 1) : sq.len - 1;  // last visible key
+    // Last visible key of this row (-1: none) and whether the row is output.
+    int lim;
+    bool row_ok;
+    size_t out_row;   // row index of O / LSE in units of heads
+    if constexpr (!DEC) {
+      const int qpos = m_blk * BM + row;
+      lim = p.causal ? min(qpos, sq.len - 1) : sq.len - 1;
+      row_ok = qpos < sq.len;
+      out_row = static_cast<size_t>(sq.start + qpos) * p.H + h;
+    } else {
+      // Row r is query token r / g (position len - q_len + r / g of the
+      // sequence) of query head hk * g + r % g.
+      row_ok = row < dec.n_rows;
+      const int pos = sq.len - dec.q_len + row / dec.g;
+      lim = !row_ok ? -1 : (p.causal ? min(pos, sq.len - 1) : sq.len - 1);
+      out_row = static_cast<size_t>(b * dec.q_len + row / dec.g) * p.H + hk * dec.g + row % dec.g;
+    }
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float c2 = p.scale_log2;
     float* mref_s = reinterpret_cast<float*>(smem + C::OFF_MREF);
@@ -317,7 +448,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t w[32];
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((k16 ^ (row & 7)) << 4));
+            // Decode rows past the q_len x g block were never loaded: zeros.
+            const uint4 v = (DEC && !row_ok)
+                                ? make_uint4(0, 0, 0, 0)
+                                : *reinterpret_cast<const uint4*>(rowp + ((k16 ^ (row & 7)) << 4));
             w[4 * k16 + 0] = v.x;
             w[4 * k16 + 1] = v.y;
             w[4 * k16 + 2] = v.z;
@@ -351,7 +485,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       mbar_arrive(bars.s_free(g));
 
-      const int nvalid = lim - j * BN + 1;  // visible keys in this tile
+      const int nvalid = lim - (j0 + j) * BN + 1;  // visible keys in this tile
       if (nvalid < BN) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -452,9 +586,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (m_g != -INFINITY) l += (m_g == m_fin) ? l_g : l_g * ex2_approx(m_g - m_fin);
       if (m_o != -INFINITY) l += (m_o == m_fin) ? l_o : l_o * ex2_approx(m_o - m_fin);
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const bool store = qpos < sq.len;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) +
-                            (static_cast<size_t>(sq.start + qpos) * p.H + h) * D;
+      const float lse = (l > 0.f) ? (m_fin + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      // Split partials (decode with several splits) stay fp32 for the merge.
+      const bool part = DEC && dec.n_split > 1;
+      const size_t prow = static_cast<size_t>(split) * p.total * p.H + out_row;
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
         const int c = g * (D / 64) + cc;   // this group's 32-column chunks
@@ -462,8 +597,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
         tmem_ld_wait();
         reg_fence(o);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        if (row_ok && part) {
+          float4* dst = reinterpret_cast<float4*>(dec.o_part + prow * D + 32 * c);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            dst[v4] = make_float4(__uint_as_float(o[4 * v4 + 0]) * inv_l,
+                                  __uint_as_float(o[4 * v4 + 1]) * inv_l,
+                                  __uint_as_float(o[4 * v4 + 2]) * inv_l,
+                                  __uint_as_float(o[4 * v4 + 3]) * inv_l);
+        } else if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + out_row * D +
+                                                32 * c);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 w;
@@ -475,9 +619,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (store && g == 0) {
-        const float lse = (l > 0.f) ? (m_fin + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-        p.lse[lse_index(p, b, h, sq.start, qpos)] = lse;
+      if (row_ok && g == 0) {
+        if constexpr (!DEC)
+          p.lse[lse_index(p, b, h, sq.start, m_blk * BM + row)] = lse;
+        else if (part)
+          dec.lse_part[prow] = lse;
+        else
+          p.lse[out_row] = lse;
       }
     }
   }
@@ -488,6 +636,45 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+}
+
+// Merge of the split partials of one output row per warp: LSE = ln sum_s
+// exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s (agentalpha.top "flash attention"
+// answer, follow-up 2: the splits are merged with the online-softmax update).
+template <int D>
+__global__ void __launch_bounds__(256)
+    decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse, long long rows,
+                          int n_split) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  float m = -INFINITY;
+  for (int s = lane; s < n_split; s += 32) m = fmaxf(m, lse_part[s * rows + row]);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, d));
+  constexpr int PER = D / 32;   // columns per lane
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  float tot = 0.f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < n_split; ++s) {
+      const float ls = lse_part[s * rows + row];
+      if (ls == -INFINITY) continue;
+      const float w = expf(ls - m);
+      tot += w;
+      const float* src = o_part + (s * rows + row) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] += w * src[i];
+    }
+  }
+  const float inv = (tot > 0.f) ? 1.f / tot : 0.f;
+  __nv_bfloat16* dst = o + row * D + lane * PER;
+#pragma unroll
+  for (int i = 0; i < PER; i += 2)
+    *reinterpret_cast<uint32_t*>(dst + i) = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+  if (lane == 0) lse[row] = (tot > 0.f) ? m + logf(tot) : -INFINITY;
 }
 
 template <int D>
@@ -502,12 +689,40 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
       !make_tmap_bf16_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN) ||
       !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int group = l2_group(4ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_bf16_kernel<D><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(tq, tk, tv, p,
-                                                                                 num_m, group);
+  fwd_bf16_kernel<D, false><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, num_m, group, DecodeArgs{});
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  const long long ctas = static_cast<long long>(p.B) * p.H_kv * d.n_split;
+  if (ctas == 0) return cudaSuccess;
+  if (ctas > INT_MAX) return cudaErrorInvalidConfiguration;
+  CUtensorMap tq, tk, tv;
+  const unsigned box_rows = (d.block_table != nullptr) ? static_cast<unsigned>(min(d.page, BN)) : BN;
+  if (!make_tmap_bf16_3d(&tq, p.q, p.total, p.H, D, static_cast<unsigned>(d.g),
+                         static_cast<unsigned>(d.q_len)) ||
+      !make_tmap_bf16_2d(&tk, p.k, d.cache_rows, static_cast<unsigned long long>(p.H_kv) * D, 64,
+                         box_rows) ||
+      !make_tmap_bf16_2d(&tv, p.v, d.cache_rows, static_cast<unsigned long long>(p.H_kv) * D, 64,
+                         box_rows))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  fwd_bf16_kernel<D, true><<<static_cast<unsigned>(ctas), THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, 0, 0, d);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || d.n_split == 1) return e;
+  const long long rows = p.total * p.H;
+  decode_combine_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      d.o_part, d.lse_part, static_cast<__nv_bfloat16*>(p.o), p.lse, rows, d.n_split);
   return cudaGetLastError();
 }
 
@@ -516,6 +731,12 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
 cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream) {
   if (p.D == 64) return launch_d<64>(p, stream);
   if (p.D == 128) return launch_d<128>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_bf16(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream) {
+  if (p.D == 64) return launch_decode_d<64>(p, d, stream);
+  if (p.D == 128) return launch_decode_d<128>(p, d, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -94,6 +94,25 @@ inline int l2_group(long long bytes_per_unit, int share, int units) {
   return static_cast<int>(g < units ? g : units);
 }
 
+// Split-KV decode (the forward kernel's decode instantiation). The queries
+// are the q_len newest tokens of each of B sequences (``AttnParams::q`` /
+// ``o`` are [B*q_len, H, D], ``total`` = B*q_len, ``max_seqlen`` bounds the
+// cache lengths); ``k`` / ``v`` point at the caches [cache_rows, H_kv, D].
+struct DecodeArgs {
+  const int* cache_seqlens;  // [B] keys of each sequence
+  const int* block_table;    // [B, max_blocks] page ids, or null: contiguous cache
+  int page;                  // paged: rows per page; contiguous: rows per sequence
+  int max_blocks;            // block-table row length
+  long long cache_rows;      // rows of k / v
+  int q_len;                 // query tokens per sequence
+  int g;                     // query heads per key/value head
+  int n_rows;                // q_len * g rows of one CTA's Q tile (<= 128)
+  int n_split;               // key splits per (sequence, kv head)
+  int chunk;                 // 128-key tiles per split
+  float* o_part;             // [n_split, B*q_len, H, D] fp32 (n_split > 1)
+  float* lse_part;           // [n_split, B*q_len, H] fp32 (n_split > 1)
+};
+
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const AttnParams& p, cudaStream_t stream);
@@ -101,6 +120,8 @@ cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream);
 // mask: bit 0 preprocess (D_i), bit 1 dK/dV kernel, bit 2 dQ kernel.
 cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned mask);
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
+// Decode partials (and the combine kernel when d.n_split > 1).
+cudaError_t launch_decode_bf16(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream);
 
 // Host: cuTensorMapEncodeTiled through the runtime's driver entry point.
 // Encodes a 2-D bf16 view [rows, cols] (row stride ``cols`` elements) with a
@@ -109,9 +130,9 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long ro
                        unsigned long long cols, unsigned box_cols, unsigned box_rows);
 
 // Host: 3-D bf16 view (D, heads, rows) of a token-major [rows, heads, D]
-// tensor with a (64, 1, box_rows) box and 128-byte swizzle. Column blocks at
-// x >= D lie outside the tensor and arrive as zeros.
+// tensor with a (64, box_heads, box_rows) box and 128-byte swizzle. Column
+// blocks at x >= D lie outside the tensor and arrive as zeros.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
-                       unsigned box_rows);
+                       unsigned box_heads, unsigned box_rows);
 
 }  // namespace fa

@@ -220,6 +220,80 @@ void fa_set_wait_budget(long long cycles);
  */
 fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream);
 
+/*
+ * ---------------------------------------------------------------- decode ---
+ * Split-KV decode (FlashDecoding) over a contiguous or paged key/value cache.
+ *
+ * At inference the method keeps its tiling and drops recomputation
+ * (agentalpha.top "flash attention" answer, section 2). The cache is split
+ * into blocks whose attention is computed independently and merged with the
+ * online-softmax update; a paged cache is read page by page (same answer,
+ * follow-up 2). Result: attention of the q_len newest tokens of each of B
+ * sequences against that sequence's cache prefix. The query token i of q_len
+ * sits at position cache_seqlens[b] - q_len + i. With causal = 1 it sees keys
+ * at positions <= its own; with causal = 0 it sees the whole prefix. A token
+ * that sees no key (for instance when cache_seqlens[b] == 0) gets O = 0 and
+ * LSE = -inf.
+ *
+ * fa_decode_num_splits - number of key splits fa_decode uses: ``requested``
+ * when > 0, else a count aiming at about four CTAs per SM of a 148-SM B200.
+ * In both cases it is clamped to the 128-key tiles of max_seqlen_k and then
+ * to the fewest splits with the same tiles per split. Host only.
+ */
+int fa_decode_num_splits(int B, int H_kv, int max_seqlen_k, int requested);
+
+/*
+ * fa_decode_workspace_size - bytes of device workspace fa_decode needs for
+ * these sizes and split request: 0 when it uses one split; otherwise fp32
+ * split partials of O and LSE (n_split * B * q_len * H * (D + 1) * 4 bytes,
+ * each array rounded up to 256 bytes). Host only. Returns 0 for invalid
+ * sizes as well; fa_decode reports those.
+ */
+size_t fa_decode_workspace_size(int B, int q_len, int H, int H_kv, int D, int max_seqlen_k,
+                                int n_split);
+
+/*
+ * fa_decode - bf16 split-KV decode attention.
+ *   q             bf16 [B * q_len, H, D], token-major: the q_len newest tokens
+ *                 of sequence b are rows b * q_len .. b * q_len + q_len - 1.
+ *   k_cache,      bf16 [cache_rows, H_kv, D] each.
+ *   v_cache       Contiguous cache (block_table NULL): position j of sequence
+ *                 b is row b * page_size + j, so page_size is the rows per
+ *                 sequence (>= max_seqlen_k). Paged cache: position j is row
+ *                 block_table[b * max_blocks + j / page_size] * page_size +
+ *                 j % page_size. Rows no position of a sequence maps to may
+ *                 hold anything (NaN included); they never reach O.
+ *   o             bf16 [B * q_len, H, D] out.
+ *   lse           fp32 [B * q_len, H] out: natural-log LSE of the scaled
+ *                 logits, -inf for a token that sees no key.
+ *   cache_seqlens device int32 [B]: keys in each sequence's cache, each in
+ *                 [0, max_seqlen_k] (a value outside is reported by
+ *                 fa_check_device_error and that sequence is left unwritten).
+ *   block_table   device int32 [B, max_blocks] page ids (entries past a
+ *                 sequence's last page are never read), or NULL.
+ *   page_size     paged: rows per page, a multiple of 16 that divides 128 or
+ *                 is a multiple of 128; contiguous: rows per sequence.
+ *   max_blocks    paged: row length of block_table (>= ceil(max_seqlen_k /
+ *                 page_size)); ignored when block_table is NULL.
+ *   cache_rows    rows of k_cache / v_cache (>= 1 and < 2^31; paged: a multiple of
+ *                 page_size; contiguous: >= (B - 1) * page_size + max_seqlen_k).
+ *   max_seqlen_k  host-side bound on cache_seqlens.
+ *   H, H_kv       query / key-value heads, H % H_kv == 0. The q_len tokens x
+ *                 H / H_kv query heads that share a key/value head form one
+ *                 128-row tile: q_len * (H / H_kv) <= 128.
+ *   D             64 or 128. scale <= 0 means 1 / sqrt(D).
+ *   n_split       key splits (0: automatic, see fa_decode_num_splits).
+ *   workspace     device, 16-byte aligned, ws_bytes >=
+ *                 fa_decode_workspace_size(...) (may be NULL when that is 0).
+ * Ownership, stream and errors as for fa_fwd: nothing is allocated; argument
+ * errors return FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED before any launch.
+ */
+fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                    const int* cache_seqlens, const int* block_table, int B, int q_len, int H,
+                    int H_kv, int D, int page_size, int max_blocks, long long cache_rows,
+                    int max_seqlen_k, int causal, float scale, int n_split, void* workspace,
+                    size_t ws_bytes, fa_stream_t stream);
+
 /* fa_version - library version as major * 10000 + minor * 100 + patch. */
 int fa_version(void);
 

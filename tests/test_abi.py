@@ -110,3 +110,51 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no non-CUDA fallback"):
         _abi.lib()
+
+
+# ------------------------------------------------------------------ decode ---
+
+def _decode(lib, **kw):
+    a = dict(q=None, k=None, v=None, o=None, lse=None, lens=None, table=None, B=2, q_len=1, H=8,
+             H_kv=2, D=128, page=1024, max_blocks=0, rows=2048, max_len=1000, causal=1,
+             scale=-1.0, n_split=0, ws=None, ws_bytes=0)
+    a.update(kw)
+    return lib.fa_decode(a["q"], a["k"], a["v"], a["o"], a["lse"], a["lens"], a["table"], a["B"],
+                         a["q_len"], a["H"], a["H_kv"], a["D"], a["page"], a["max_blocks"],
+                         a["rows"], a["max_len"], a["causal"], a["scale"], a["n_split"], a["ws"],
+                         a["ws_bytes"], None)
+
+
+def test_decode_rejects_bad_shapes_before_any_launch(lib):
+    assert _decode(lib, D=96) == _abi.FA_ERR_UNSUPPORTED
+    assert _decode(lib, q_len=17, H=64, H_kv=8) == _abi.FA_ERR_UNSUPPORTED   # 136 rows > 128
+    assert _decode(lib, H=6, H_kv=4) == _abi.FA_ERR_INVALID_ARG
+    assert _decode(lib, q_len=0) == _abi.FA_ERR_INVALID_ARG
+    assert _decode(lib, page=999) == _abi.FA_ERR_INVALID_ARG       # stride < max_seqlen_k
+    assert _decode(lib, rows=1500) == _abi.FA_ERR_INVALID_ARG      # contiguous cache too short
+    assert _decode(lib, rows=0) == _abi.FA_ERR_INVALID_ARG
+    assert _decode(lib, rows=1 << 31) == _abi.FA_ERR_UNSUPPORTED
+    fake = ctypes.c_void_p(16)
+    assert _decode(lib, table=fake, page=48, max_blocks=64) == _abi.FA_ERR_UNSUPPORTED
+    assert _decode(lib, table=fake, page=64, max_blocks=15) == _abi.FA_ERR_INVALID_ARG
+    assert _decode(lib, table=fake, page=64, max_blocks=16, rows=2000) == _abi.FA_ERR_INVALID_ARG
+    # null tensors with otherwise valid sizes
+    assert _decode(lib) == _abi.FA_ERR_INVALID_ARG
+    assert _decode(lib, B=0) == _abi.FA_OK
+
+
+def test_decode_split_count_and_workspace_size(lib):
+    # automatic: about 4 * 148 CTAs over B * H_kv units, clamped to the tiles
+    assert lib.fa_decode_num_splits(16, 8, 32768, 0) == 5     # ceil(592 / 128) = 5 of 256 tiles
+    assert lib.fa_decode_num_splits(1, 1, 1000, 0) == 8       # clamped to 8 tiles
+    assert lib.fa_decode_num_splits(2, 2, 1000, 3) == 3       # chunk 3 -> 3 splits
+    assert lib.fa_decode_num_splits(2, 2, 1000, 7) == 4       # chunk 2 -> 4 splits
+    assert lib.fa_decode_num_splits(2, 2, 0, 0) == 1
+    assert lib.fa_decode_workspace_size(2, 1, 8, 2, 128, 1000, 1) == 0
+    ns = lib.fa_decode_num_splits(2, 2, 1000, 3)
+    rows = ns * 2 * 1 * 8
+
+    def r256(x):
+        return (x + 255) // 256 * 256
+    assert lib.fa_decode_workspace_size(2, 1, 8, 2, 128, 1000, 3) == r256(rows * 128 * 4) + \
+        r256(rows * 4)
