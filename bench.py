@@ -9,6 +9,11 @@ synthetic Gaussians resident in HBM before the timed region starts.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the float64 CPU oracle arm)
 
+A decode workload (``--workload bf16_decode_...``) times the split-KV decode
+path instead: a step is one fa_decode call (split partials + merge) of the
+q_len newest tokens of every sequence against its KV cache, resident in HBM;
+the metric is the KV-cache bytes it must read per second.
+
 With N > 1 (launched by torch.distributed.run) every rank runs its own
 independently seeded batch of the same shape (the (batch, head) units are
 independent; no collective on the data path): weak scaling, timed as the
@@ -35,6 +40,8 @@ METRIC = "attention fwd/bwd TFLOP/s (bf16, device-timed) and % of B200 dense BF1
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "bf16_causal_b2_h16_n8192_d128"
 L2_BYTES = 126 * 1024 * 1024
+DECODE_METRIC = "split-KV decode attention, KV-cache GB/s read (bf16, device-timed)"
+DECODE_UNIT = "GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -89,7 +96,8 @@ def source_sha(*names) -> str:
 
 KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
-                  "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h")}
+                  "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
+                  "decode": ("fwd_bf16.cu", "common.cuh", "params.h")}
 
 
 def recorded_traffic(kernel: str, workload: str):
@@ -419,6 +427,203 @@ def run_ours(args, w) -> None:
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------- decode arm ---
+
+def decode_config(w) -> dict:
+    lengths = w.lengths()
+    return {"workload": w.name, "B": w.B, "q_len": w.q_len, "H": w.H, "H_kv": w.H_kv, "D": w.D,
+            "causal": w.causal, "cache": f"paged, {w.page_size} rows per page, shuffled blocks"
+            if w.page_size else "contiguous", "cache_len_range": [w.len_lo, w.len_hi],
+            "cache_tokens": int(sum(lengths)), "pass": "decode", "seed": w.seed}
+
+
+def decode_oracle_sample(w, n_seq: int):
+    """The float64 decode oracle on the first ``n_seq`` sequences of the
+    workload. Returns (seconds, KV bytes, FLOPs)."""
+    from exact_io_aware_tmem_b200.workloads import decode_bytes, decode_case, decode_flops
+    from oracle import decode as od
+    lengths = w.lengths()[:n_seq]
+    c = decode_case(w.seed, dtype=w.dtype, lengths=lengths, q_len=w.q_len, H=w.H, H_kv=w.H_kv,
+                    D=w.D, page_size=w.page_size)
+    t0 = time.perf_counter()
+    od.decode_forward(c.q, c.k_cache, c.v_cache, c.cache_seqlens, q_len=w.q_len, scale=w.scale,
+                      causal=w.causal, stride=c.page_size, page_size=c.page_size,
+                      block_table=c.block_table)
+    dt = time.perf_counter() - t0
+    return dt, decode_bytes(lengths, w.H_kv, w.D), decode_flops(lengths, w.q_len, w.H, w.D)
+
+
+def decode_cpu_baseline(w) -> dict:
+    n = max(1, w.B // 4)
+    dt, by, _ = decode_oracle_sample(w, n)
+    return {"value": by / dt / 1e9, "unit": DECODE_UNIT, "cores": blas_threads(),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"float64 numpy decode oracle on the first {n} of the {w.B} sequences of "
+                      f"{w.name}; bytes by the same formula as the GPU line"}
+
+
+def run_decode_reference(args, w) -> None:
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    n = max(1, w.B // 4)
+    for _ in range(args.warmup):
+        decode_oracle_sample(w, n)
+    tot_t = tot_b = 0.0
+    for _ in range(args.steps):
+        dt, by, _ = decode_oracle_sample(w, n)
+        tot_t += dt
+        tot_b += by
+    value = tot_b / tot_t / 1e9
+    sample = f"float64 numpy decode oracle, first {n} of {w.B} sequences of {w.name} per step"
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": decode_config(w),
+            "cpu_baseline": {"value": value, "unit": DECODE_UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": DECODE_UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_decode(args, w) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import exact_io_aware_tmem_b200 as fa
+    from exact_io_aware_tmem_b200.workloads import (DecodeWorkload, decode_bytes, decode_flops,
+                                                    make_decode_inputs)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    peaks = load_peaks()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = decode_cpu_baseline(w)
+
+    wr = DecodeWorkload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})
+    c = make_decode_inputs(wr)
+    lengths = c.cache_seqlens.tolist()
+    max_len = max(lengths)
+    kv_bytes = decode_bytes(lengths, w.H_kv, w.D)
+    fl = decode_flops(lengths, w.q_len, w.H, w.D)
+    q = c.q.to(dev)
+    kc, vc = c.k_cache.to(dev), c.v_cache.to(dev)
+    lens = c.cache_seqlens.to(dev)
+    table = None if c.block_table is None else c.block_table.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((q.shape[0], w.H), device=dev, dtype=torch.float32)
+    n_split = fa.decode_num_splits(w.B, w.H_kv, max_len)
+    ws = torch.empty(max(1, fa.decode_workspace_size(w.B, w.q_len, w.H, w.H_kv, w.D, max_len)),
+                     dtype=torch.uint8, device=dev)
+    alg_bytes = kv_bytes + 2 * q.numel() * q.element_size() + lse.numel() * 4
+
+    def step():
+        fa.decode(q, kc, vc, lens, q_len=w.q_len, max_seqlen_k=max_len, block_table=table,
+                  page_size=c.page_size, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                  workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    st, where = fa.check_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where:#x} during warm-up")
+    gpu_uuid = ""
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        gpu_uuid = gpu_uuid if gpu_uuid.startswith("GPU-") else "GPU-" + gpu_uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_uuid)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    start.record()
+    for i in range(args.steps):
+        evs[i][0].record()
+        step()
+        evs[i][1].record()
+    end.record()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    st, where = fa.check_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where:#x} in the timed region")
+    max_ms = reduce_max(start.elapsed_time(end), dev)
+    call_ms = reduce_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs), dev)
+
+    # End to end: the step's new tokens (Q, and the cache lengths) go host ->
+    # device from pinned memory and O, LSE come back; the KV cache is the
+    # state a decode step reads in place, resident as in serving.
+    e2e_steps = max(3, min(args.steps, 50))
+    hq, hl = q.cpu().pin_memory(), lens.cpu().pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hs = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = q.numel() * q.element_size() + lens.numel() * 4
+    d2h = o.numel() * o.element_size() + lse.numel() * 4
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record()
+    for _ in range(e2e_steps):
+        q.copy_(hq, non_blocking=True)
+        lens.copy_(hl, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hs.copy_(lse, non_blocking=True)
+    e_end.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e_start.elapsed_time(e_end), dev)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    value = aggregate(kv_bytes * args.steps, world, [max_ms / 1e3]) / 1e9
+    achieved = alg_bytes / (call_ms / 1e3) / 1e9
+    peak = peaks["hbm_gbs"]
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(decode_config(w), n_split=n_split,
+                       parallelism=f"replicas{world}" if world > 1 else "none",
+                       l2=f"not flushed: every step reads {kv_bytes / 2**20:.0f} MiB of cache "
+                          f"> {L2_BYTES >> 20} MiB L2",
+                       ranks="each rank its own seeded batch of this shape"),
+        "tflops": fl / (call_ms / 1e3) / 1e12,
+        "kernel_ms": {"fa_decode (partials + merge)": round(call_ms, 4)},
+        "roofline": {"kernel": "fwd_bf16_kernel<decode> + decode_combine_kernel (one fa_decode)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peaks['source']} HBM copy",
+                     "algorithmic_bytes": alg_bytes,
+                     "traffic": recorded_traffic("decode", w.name)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": kv_bytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9,
+                "unit": DECODE_UNIT, "steps": e2e_steps, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": (2 if n_split > 1 else 1) * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -429,10 +634,17 @@ def main(argv=None) -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
-    from exact_io_aware_tmem_b200.workloads import WORKLOADS
-    w = WORKLOADS[args.workload]
+    from exact_io_aware_tmem_b200.workloads import DECODE_WORKLOADS, WORKLOADS
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in DECODE_WORKLOADS:
+        w = DECODE_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            run_decode_reference(args, w)
+        else:
+            run_decode(args, w)
+        return 0
+    w = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
     else:

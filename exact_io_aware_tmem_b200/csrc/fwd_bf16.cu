@@ -237,29 +237,73 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == WARP_TMA) {
     // ------------------------------------------------------ TMA producer ---
-    // K / V tile jt (absolute key tile) into shared memory at ``dst``.
-    auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int jt) {
-      if constexpr (!DEC) {
-#pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, sq.start + jt * BN);
-      } else if (dec.block_table == nullptr) {
-        const int row = b * dec.page + jt * BN;
-#pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, row);
+    // The whole warp runs the producer loop; lane 0 issues the copies.
+    //
+    // Paged cache: the page ids a stream (K or V) needs are read 32 at a
+    // time, one coalesced load per batch, lane L holding page base + L, with
+    // the next batch already in flight; a tile's ids then come by shuffle.
+    // Looking each id up on its own put an L2 round trip in front of every
+    // TMA issue. -1: a page past the sequence's end (or past the table row).
+    const int n_pages = DEC ? (sq.len + dec.page - 1) / max(dec.page, 1) : 0;
+    auto page_id = [&](int pg) -> int {
+      if constexpr (DEC) {
+        return (pg < n_pages && pg < dec.max_blocks)
+                   ? __ldg(dec.block_table + static_cast<size_t>(b) * dec.max_blocks + pg)
+                   : -1;
       } else {
-        // Paged: one box per page (or one 128-row box inside a larger page).
-        // Pages past the sequence's end load from beyond the cache: zeros.
-        const int box = min(dec.page, BN);
-        for (int u = 0; u < BN / box; ++u) {
-          const int key = jt * BN + u * box;
+        return -1;
+      }
+    };
+    struct PageBatch {
+      int base, cur, nxt;
+    };
+    auto batch_init = [&](PageBatch& pb, int first) {
+      pb.base = first;
+      pb.cur = page_id(first + lane);
+      pb.nxt = page_id(first + 32 + lane);
+    };
+    // Page id of page pg0 + min(lane, n - 1): the n (<= 8) pages of one tile,
+    // one per lane. pg0 is warp-uniform and never decreases.
+    auto batch_get = [&](PageBatch& pb, int pg0, int n) -> int {
+      while (pg0 >= pb.base + 32) {
+        pb.base += 32;
+        pb.cur = pb.nxt;
+        pb.nxt = page_id(pb.base + 32 + lane);
+      }
+      const int off = pg0 + min(lane, n - 1) - pb.base;   // < 32 + 8
+      const int from_cur = __shfl_sync(FULL, pb.cur, off & 31);
+      const int from_nxt = __shfl_sync(FULL, pb.nxt, off & 31);
+      return off < 32 ? from_cur : from_nxt;
+    };
+    const bool paged = DEC && dec.block_table != nullptr;
+    const int box = paged ? min(dec.page, BN) : BN;   // rows per TMA box
+    // K / V tile jt (absolute key tile) into shared memory at ``dst``. The
+    // caller has posted the tile's expected bytes on ``bar``.
+    auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int jt, PageBatch& pb) {
+      if constexpr (!DEC) {
+        if (lane == 0) {
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, sq.start + jt * BN);
+        }
+      } else if (!paged) {
+        if (lane == 0) {
+          const int row = b * dec.page + jt * BN;
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, row);
+        }
+      } else {
+        // One box per page (or one 128-row box inside a larger page), lane u
+        // issuing page u's box so small pages do not serialise on one
+        // thread. Pages past the sequence's end load from beyond the cache:
+        // zeros.
+        const int n = BN / box;
+        const int blk = batch_get(pb, jt * BN / dec.page, n);
+        if (lane < n) {
+          const int key = jt * BN + lane * box;
           int row = static_cast<int>(dec.cache_rows);
           if (key < sq.len) {
-            const int pg = key / dec.page;
-            const int blk = (pg < dec.max_blocks)
-                                ? __ldg(dec.block_table + static_cast<size_t>(b) * dec.max_blocks + pg)
-                                : -1;
             if (blk >= 0 && static_cast<long long>(blk + 1) * dec.page <= dec.cache_rows)
               row = blk * dec.page + key % dec.page;
             else
@@ -267,7 +311,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_2d(dst + c * CHUNK_BYTES + u * box * 128, map, bar, hk * D + c * 64, row);
+            tma_load_2d(dst + c * CHUNK_BYTES + lane * box * 128, map, bar, hk * D + c * 64, row);
         }
       }
     };
@@ -289,40 +333,55 @@ __global__ void __launch_bounds__(THREADS, 1)
           tma_load_3d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), c * 64, hk * dec.g,
                       b * dec.q_len);
       }
-      // K and V run through separate rings and are loaded independently, K
-      // first whenever both have a free slot: K_j is consumed early (QK_j
-      // runs two tiles ahead of PV_j), and a K load that waited behind a V
-      // slot would stall the score MMAs on the slowest event of the loop.
-      int jk = 0, jv = 0;
-      long long t_last = clock64();
-      while (jk < n_kv || jv < n_kv) {
-        bool progress = false;
-        if (jk < n_kv && mbar_try_wait(bars.k_empty(jk % C::STAGES),
-                                       ((jk / C::STAGES) & 1) ^ 1)) {
-          const int st = jk % C::STAGES;
-          mbar_arrive_expect_tx(bars.k_full(st), C::TILE);
-          load_kv(sbase + C::OFF_K + st * C::TILE, &tm_k, bars.k_full(st), j0 + jk);
-          ++jk;
-          progress = true;
-        }
-        if (jv < n_kv && jv < jk &&
-            mbar_try_wait(bars.v_empty(jv % C::STAGES), ((jv / C::STAGES) & 1) ^ 1)) {
-          const int st = jv % C::STAGES;
-          mbar_arrive_expect_tx(bars.v_full(st), C::TILE);
-          load_kv(sbase + C::OFF_V + st * C::TILE, &tm_v, bars.v_full(st), j0 + jv);
-          ++jv;
-          progress = true;
-        }
-        if (progress) {
-          t_last = clock64();
-        } else if (*abort) {
-          break;
-        } else if (clock64() - t_last > p.err.budget) {
+    }
+    // K and V run through separate rings and are loaded independently, K
+    // first whenever both have a free slot: K_j is consumed early (QK_j runs
+    // two tiles ahead of PV_j), and a K load that waited behind a V slot
+    // would stall the score MMAs on the slowest event of the loop.
+    PageBatch kpb{0, -1, -1}, vpb{0, -1, -1};
+    if (paged) {
+      batch_init(kpb, j0 * BN / dec.page);
+      batch_init(vpb, j0 * BN / dec.page);
+    }
+    int jk = 0, jv = 0;
+    long long t_last = clock64();
+    while (jk < n_kv || jv < n_kv) {
+      bool progress = false;
+      if (jk < n_kv &&
+          __all_sync(FULL, mbar_try_wait(bars.k_empty(jk % C::STAGES),
+                                         ((jk / C::STAGES) & 1) ^ 1))) {
+        const int st = jk % C::STAGES;
+        if (lane == 0) mbar_arrive_expect_tx(bars.k_full(st), C::TILE);
+        __syncwarp();
+        load_kv(sbase + C::OFF_K + st * C::TILE, &tm_k, bars.k_full(st), j0 + jk, kpb);
+        ++jk;
+        progress = true;
+      }
+      if (jv < jk &&
+          __all_sync(FULL, mbar_try_wait(bars.v_empty(jv % C::STAGES),
+                                         ((jv / C::STAGES) & 1) ^ 1))) {
+        const int st = jv % C::STAGES;
+        if (lane == 0) mbar_arrive_expect_tx(bars.v_full(st), C::TILE);
+        __syncwarp();
+        load_kv(sbase + C::OFF_V + st * C::TILE, &tm_v, bars.v_full(st), j0 + jv, vpb);
+        ++jv;
+        progress = true;
+      }
+      if (progress) {
+        t_last = clock64();
+        continue;
+      }
+      // Lane 0 decides, so the whole warp leaves the loop together.
+      const int stop =
+          __shfl_sync(FULL, *abort ? 1 : (clock64() - t_last > p.err.budget ? 2 : 0), 0);
+      if (stop == 1) break;
+      if (stop == 2) {
+        if (lane == 0) {
           *abort = 1;
           atomicOr(p.err.word, ERR_TIMEOUT);
           atomicExch(p.err.word + 1, jk < n_kv ? W_KEMPTY : W_VEMPTY);
-          break;
         }
+        break;
       }
     }
     if (v_tail) {
