@@ -527,11 +527,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       // group 1 writes none before group 0 has finished copying Q out of it.
       ok = warp_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM);
     }
+    // Decode warps whose 32 rows are all padding (q_len x g < 128) keep the
+    // barrier protocol - the same waits and arrivals, in the same order, so
+    // no barrier phase ever mixes two tiles - but load, exponentiate and
+    // store nothing: their rows are never written out.
+    const bool idle = DEC && __all_sync(FULL, !row_ok);
     for (int j = g; j < n_kv && ok; j += 2) {
       const uint32_t s_col = TM_S0 + g * BN;
       if (!warp_wait(bars.s_full(g), (j >> 1) & 1, p.err, abort, W_SFULL)) {
         ok = false;
         break;
+      }
+      if (idle) {
+        mbar_arrive(bars.s_free(g));
+        if (j > 0 && !warp_wait(bars.mref(g ^ 1), ((j - 1) >> 1) & 1, p.err, abort, W_MREF)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive(bars.mref(g));
+        if (j > 0 &&
+            !warp_wait(bars.pv_done(g ^ 1), ((j - 1) >> 1) & 1, p.err, abort, W_PVDONE)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive(bars.p_ready());
+        continue;
       }
       tc_fence_after();
       uint32_t r[4][32];
@@ -636,7 +656,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = warp_wait(bars.fin(), 0, p.err, abort, W_FIN);
     }
     const int last = n_kv - 1;
-    if (ok && warp_wait(bars.pv_done(last & 1), (last >> 1) & 1, p.err, abort, W_PVDONE)) {
+    if (ok && !idle &&
+        warp_wait(bars.pv_done(last & 1), (last >> 1) & 1, p.err, abort, W_PVDONE)) {
       tc_fence_after();
       const float m_o = fin_s[(2 * (g ^ 1)) * BM + row];
       const float l_o = fin_s[(2 * (g ^ 1) + 1) * BM + row];
