@@ -50,6 +50,10 @@ SIGNATURES = {
     "fa_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                           c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_ll, c_int, c_int,
                           c_float, c_int, c_void_p, c_size_t, c_void_p]),
+    "fa_fp8_quantize": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                                c_void_p]),
+    "fa_fwd_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                           c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_void_p]),
     "fa_version": (c_int, []),
 }
 

@@ -153,6 +153,35 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     return out, lse
 
 
+def fp8_quantize(x: torch.Tensor, B: int, N: int):
+    """Pass 1 of the FP8 forward: E4M3 codes (uint8, x's shape) and per-block
+    steps fp32 [B, Hx, ceil(N / 128)] of a bf16 [B*N, Hx, D] (or [B, N, Hx, D]) tensor."""
+    Hx, D = x.shape[-2], x.shape[-1]
+    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sc = torch.empty((B, Hx, (N + 127) // 128), dtype=torch.float32, device=x.device)
+    st = _abi.lib().fa_fp8_quantize(_ptr(x), _ptr(x8), _ptr(sc), B, N, Hx, D, _stream(x.device))
+    _abi.check(st, "fa_fp8_quantize")
+    return x8, sc
+
+
+def fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v: torch.Tensor, q_scale: torch.Tensor,
+            k_scale: torch.Tensor, *, B: int, N: int, causal: bool = False,
+            scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None):
+    """Pass 2 of the FP8 forward (fa_fwd_fp8). Returns (O bf16, LSE [B, H, N])."""
+    H, D = q8.shape[-2], q8.shape[-1]
+    H_kv = k8.shape[-2]
+    if out is None:
+        out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    st = _abi.lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(q_scale), _ptr(k_scale),
+                               _ptr(out), _ptr(lse), B, H, H_kv, N, D, int(bool(causal)),
+                               -1.0 if scale is None else float(scale), _stream(q8.device))
+    _abi.check(st, "fa_fwd_fp8")
+    return out, lse
+
+
 def check_device_error(device: Optional[torch.device] = None) -> tuple:
     """Synchronise the current stream; return (status, where) and clear the flag."""
     import ctypes

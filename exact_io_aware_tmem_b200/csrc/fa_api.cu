@@ -124,6 +124,19 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long ro
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, unsigned long long rows,
+                     unsigned long long cols, unsigned box_cols, unsigned box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};  // bytes between rows
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D,
                        unsigned box_heads, unsigned box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -290,6 +303,42 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, voi
   }
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return fa::cuda_status(fa::launch_decode_bf16(p, d, s));
+}
+
+fa_status fa_fp8_quantize(const void* x, void* x8, float* scale, int B, int N, int Hx, int D,
+                          fa_stream_t stream) {
+  if (B < 0 || N < 0 || Hx <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 256) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * N > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!x || !x8 || !scale) return FA_ERR_INVALID_ARG;
+  if (!fa::aligned16(x) || !fa::aligned16(x8)) return FA_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return fa::cuda_status(fa::launch_fp8_quantize(x, x8, scale, B, N, Hx, D, s));
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v, const float* q_scale,
+                     const float* k_scale, void* o, float* lse, int B, int H, int H_kv, int N,
+                     int D, int causal, float scale, fa_stream_t stream) {
+  AttnParams p = {};
+  fa_status st = fa::check_common(p, B, H, H_kv, N, D, FA_BF16, causal, scale, nullptr, N,
+                                  static_cast<long long>(B) * N);
+  if (st != FA_OK) return st;
+  if (D != 128) return FA_ERR_UNSUPPORTED;
+  if (p.total == 0 || B == 0) return FA_OK;
+  if (!q8 || !k8 || !v || !q_scale || !k_scale || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!fa::aligned16(q8) || !fa::aligned16(k8) || !fa::aligned16(v) || !fa::aligned16(o))
+    return FA_ERR_INVALID_ARG;
+  p.q = q8;
+  p.k = k8;
+  p.v = v;
+  p.o = o;
+  p.lse = lse;
+  p.err.word = fa::err_word();
+  if (p.err.word == nullptr) return FA_ERR_CUDA;
+  fa::Fp8Args f = {q_scale, k_scale, (N + 127) / 128};
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return fa::cuda_status(fa::launch_fwd_fp8(p, f, s));
 }
 
 size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype) {

@@ -73,25 +73,33 @@ enum : unsigned {
   W_VTAIL = 0x10E00, BAD_CACHE_LEN = 0x10F01, BAD_PAGE = 0x10F02
 };
 
-template <int D>
+// F8: Q and K are E4M3 tiles (one 128-byte row per token at D = 128) that
+// the score MMA reads from shared memory; V stays bf16.
+template <int D, bool F8>
 struct FwdCfg {
-  static constexpr int STAGES = (D == 64) ? 4 : 3;
-  static constexpr int CHUNKS = D / 64;
-  static constexpr uint32_t TILE = BM * D * 2;  // bytes of one 128-row tile
+  static_assert(!F8 || D == 128, "the E4M3 path has one 128-byte row per token");
+  static constexpr int STAGES = (D == 64 || F8) ? 4 : 3;
+  static constexpr int CHUNKS = D / 64;            // 128-byte blocks of a bf16 row
+  static constexpr int QK_CHUNKS = F8 ? 1 : CHUNKS; // 128-byte blocks of a Q / K row
+  static constexpr uint32_t TILE = BM * D * 2;     // bytes of one bf16 128-row tile
+  static constexpr uint32_t QK_TILE = F8 ? BM * D : TILE;
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + TILE;
-  static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
-  static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
+  static constexpr uint32_t OFF_K = OFF_Q + QK_TILE;
+  static constexpr uint32_t OFF_V = OFF_K + STAGES * QK_TILE;
+  // Per-row exchange words: reference max per group [2][128], then final
+  // (m, l) per group [2][2][128]. The bf16 paths keep them in the Q tile
+  // once Q is in TMEM; the E4M3 path reads Q from shared memory throughout.
+  static constexpr uint32_t XCHG = 6 * BM * 4;
+  static constexpr uint32_t OFF_X = F8 ? OFF_V + STAGES * TILE : OFF_Q;
+  static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE + (F8 ? XCHG : 0);
   // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
   // mref[2], pv_done[2], p_ready, q_tmem, fin, v_fix
   static constexpr int NBAR = 1 + 4 * STAGES + 12;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
-  // Once Q is in TMEM its shared tile holds the per-row exchange words:
-  // reference max per group [2][128], then final (m, l) per group [2][2][128].
-  static constexpr uint32_t OFF_MREF = OFF_Q;
-  static constexpr uint32_t OFF_FIN = OFF_Q + 2 * BM * 4;
-  static_assert(OFF_FIN + 4 * BM * 4 <= TILE, "exchange words fit in the Q tile");
+  static constexpr uint32_t OFF_MREF = OFF_X;
+  static constexpr uint32_t OFF_FIN = OFF_X + 2 * BM * 4;
+  static_assert(F8 || XCHG <= QK_TILE, "exchange words fit in the Q tile");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -130,13 +138,17 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
 // split); its Q tile is the q_len newest tokens x the g query heads of the kv
 // head (rows r = token * g + head), and it writes that split's partial O / l
 // and LSE (or the final O and LSE when there is one split).
-template <int D, bool DEC>
+// F8 = true: Q and K arrive as E4M3 codes with one fp32 step per 128-token
+// block (pass 1, fp8.cu); S = Q_hat K_hat^T runs as a kind::f8f6f4 MMA with
+// fp32 accumulation and is scaled by Delta_Q Delta_K of its two blocks.
+template <int D, bool DEC, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m,
-                    int group, const DecodeArgs dec) {
-  using C = FwdCfg<D>;
+                    int group, const DecodeArgs dec, const Fp8Args f8) {
+  static_assert(!(DEC && F8), "the E4M3 path is a forward over dense batches");
+  using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -279,8 +291,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int box = paged ? min(dec.page, BN) : BN;   // rows per TMA box
     // K / V tile jt (absolute key tile) into shared memory at ``dst``. The
     // caller has posted the tile's expected bytes on ``bar``.
-    auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int jt, PageBatch& pb) {
-      if constexpr (!DEC) {
+    auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int jt, PageBatch& pb,
+                       bool is_k) {
+      if constexpr (F8) {
+        // E4M3 K: one 128-byte (128-code) column block; V: bf16 as below.
+        if (lane == 0) {
+          const int chunks = is_k ? 1 : C::CHUNKS;
+          for (int c = 0; c < chunks; ++c)
+            tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, sq.start + jt * BN);
+        }
+      } else if constexpr (!DEC) {
         if (lane == 0) {
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c)
@@ -321,9 +341,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&tm_v);
       if constexpr (!DEC) {
         const int row_q = sq.start + m_blk * BM;
-        mbar_arrive_expect_tx(bars.q(), C::TILE);
+        mbar_arrive_expect_tx(bars.q(), C::QK_TILE);
 #pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
+        for (int c = 0; c < C::QK_CHUNKS; ++c)
           tma_load_2d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), h * D + c * 64, row_q);
       } else {
         // q_len tokens x g heads: one (64, g, q_len) box per column block.
@@ -351,9 +371,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           __all_sync(FULL, mbar_try_wait(bars.k_empty(jk % C::STAGES),
                                          ((jk / C::STAGES) & 1) ^ 1))) {
         const int st = jk % C::STAGES;
-        if (lane == 0) mbar_arrive_expect_tx(bars.k_full(st), C::TILE);
+        if (lane == 0) mbar_arrive_expect_tx(bars.k_full(st), C::QK_TILE);
         __syncwarp();
-        load_kv(sbase + C::OFF_K + st * C::TILE, &tm_k, bars.k_full(st), j0 + jk, kpb);
+        load_kv(sbase + C::OFF_K + st * C::QK_TILE, &tm_k, bars.k_full(st), j0 + jk, kpb, true);
         ++jk;
         progress = true;
       }
@@ -363,7 +383,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int st = jv % C::STAGES;
         if (lane == 0) mbar_arrive_expect_tx(bars.v_full(st), C::TILE);
         __syncwarp();
-        load_kv(sbase + C::OFF_V + st * C::TILE, &tm_v, bars.v_full(st), j0 + jv, vpb);
+        load_kv(sbase + C::OFF_V + st * C::TILE, &tm_v, bars.v_full(st), j0 + jv, vpb, false);
         ++jv;
         progress = true;
       }
@@ -422,6 +442,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
     // Shared-memory descriptors, built once and stepped by constant offsets.
     const uint64_t k_desc = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+    const uint64_t q_desc = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);   // E4M3 path only
+    constexpr uint32_t IDESC_QK8 = idesc_e4m3(BM, BN);
     const uint64_t v_desc = sdesc_sw128(sbase + C::OFF_V, CHUNK_BYTES, 1024);
     // Q reaches TMEM through the softmax threads.
     bool ok = warp_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM);
@@ -441,11 +463,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_s = tmem + TM_S0 + (jq & 1) * BN;
+        if constexpr (F8) {
+          // M=128, N=128, K=D in steps of 32 codes (32 bytes of a row).
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-          mma_ts_if(leader, d_s, tmem + TM_Q + kk * 8, sdesc_add(k_desc, st * C::TILE + off),
-                    IDESC_QK, kk > 0);
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_ss_e4m3_if(leader, d_s, sdesc_add(q_desc, kk * 32),
+                           sdesc_add(k_desc, st * C::QK_TILE + kk * 32), IDESC_QK8, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
+            mma_ts_if(leader, d_s, tmem + TM_Q + kk * 8, sdesc_add(k_desc, st * C::QK_TILE + off),
+                      IDESC_QK, kk > 0);
+          }
         }
         tc_commit_if(leader, bars.s_full(jq & 1));
         tc_commit_if(leader, bars.k_empty(st));
@@ -490,7 +520,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       out_row = static_cast<size_t>(b * dec.q_len + row / dec.g) * p.H + hk * dec.g + row % dec.g;
     }
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float c2 = p.scale_log2;
+    float c2 = p.scale_log2;
+    // E4M3 scores are in units of Delta_Q Delta_K of their two blocks.
+    const float* kscale_row = nullptr;
+    if constexpr (F8) {
+      c2 *= __ldg(f8.q_scale + (static_cast<size_t>(b) * p.H + h) * f8.n_blocks + m_blk);
+      kscale_row = f8.k_scale + (static_cast<size_t>(b) * p.H_kv + hk) * f8.n_blocks;
+    }
     float* mref_s = reinterpret_cast<float*>(smem + C::OFF_MREF);
     float* fin_s = reinterpret_cast<float*>(smem + C::OFF_FIN);
     float m_g = -INFINITY;  // reference of this group's last tile (log2 units)
@@ -500,7 +536,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // Copy this row of Q from the swizzled shared tile into TMEM as packed
       // bf16 (even element in the low half): the A operand of S = Q K^T.
       ok = warp_wait(bars.q(), 0, p.err, abort, W_Q);
-      if (ok) {
+      if (ok && F8) {
+        mbar_arrive(bars.q_tmem());   // the E4M3 score MMA reads Q from shared memory
+      } else if (ok) {
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c) {
           const uint8_t* rowp = smem + C::OFF_Q + c * CHUNK_BYTES + row * 128;
@@ -534,6 +572,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool idle = DEC && __all_sync(FULL, !row_ok);
     for (int j = g; j < n_kv && ok; j += 2) {
       const uint32_t s_col = TM_S0 + g * BN;
+      const float c2t = F8 ? c2 * __ldg(kscale_row + j) : c2;   // log2 units per raw score
       if (!warp_wait(bars.s_full(g), (j >> 1) & 1, p.err, abort, W_SFULL)) {
         ok = false;
         break;
@@ -594,7 +633,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // The reference only moves when the row max exceeds it by more than
       // RESCALE_LOG2 (log2 units): P = 2^(s c - m_ref) then stays below
       // 2^RESCALE_LOG2, and O / l is the same for any consistent reference.
-      const float m_cand = mx * c2;
+      const float m_cand = mx * c2t;
       const bool grow = m_cand > m_prev + RESCALE_LOG2;   // always true on tile 0
       const float m_new = grow ? m_cand : m_prev;
       mref_s[g * BM + row] = m_new;
@@ -606,8 +645,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use));
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2t, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2t, -m_use));
           sum4[(i >> 1) & 3] += p0 + p1;
           pk[c >> 1][(c & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
         }
@@ -759,7 +798,7 @@ __global__ void __launch_bounds__(256)
 
 template <int D>
 cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, false>;
   const int num_m = (p.max_seqlen + BM - 1) / BM;
   const long long tiles = static_cast<long long>(num_m) * p.H * p.B;
   if (tiles == 0 || p.total == 0) return cudaSuccess;
@@ -769,18 +808,40 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
       !make_tmap_bf16_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN) ||
       !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, false>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, false, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int group = l2_group(4ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_bf16_kernel<D, false><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
-      tq, tk, tv, p, num_m, group, DecodeArgs{});
+  fwd_bf16_kernel<D, false, false><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, num_m, group, DecodeArgs{}, Fp8Args{});
+  return cudaGetLastError();
+}
+
+// E4M3 forward: p.q / p.k hold the codes, ``f`` their per-block steps.
+cudaError_t launch_fp8_d128(const AttnParams& p, const Fp8Args& f, cudaStream_t stream) {
+  constexpr int D = 128;
+  using C = FwdCfg<D, true>;
+  const int num_m = (p.max_seqlen + BM - 1) / BM;
+  const long long tiles = static_cast<long long>(num_m) * p.H * p.B;
+  if (tiles == 0 || p.total == 0) return cudaSuccess;
+  if (tiles > INT_MAX) return cudaErrorInvalidConfiguration;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_u8_2d(&tq, p.q, p.total, static_cast<unsigned long long>(p.H) * D, 128, BM) ||
+      !make_tmap_u8_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 128, BN) ||
+      !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, false, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int group = l2_group(3ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
+  fwd_bf16_kernel<D, false, true><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, num_m, group, DecodeArgs{}, f);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, false>;
   const long long ctas = static_cast<long long>(p.B) * p.H_kv * d.n_split;
   if (ctas == 0) return cudaSuccess;
   if (ctas > INT_MAX) return cudaErrorInvalidConfiguration;
@@ -793,11 +854,11 @@ cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream
       !make_tmap_bf16_2d(&tv, p.v, d.cache_rows, static_cast<unsigned long long>(p.H_kv) * D, 64,
                          box_rows))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, true>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, true, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  fwd_bf16_kernel<D, true><<<static_cast<unsigned>(ctas), THREADS, C::SMEM, stream>>>(
-      tq, tk, tv, p, 0, 0, d);
+  fwd_bf16_kernel<D, true, false><<<static_cast<unsigned>(ctas), THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, 0, 0, d, Fp8Args{});
   e = cudaGetLastError();
   if (e != cudaSuccess || d.n_split == 1) return e;
   const long long rows = p.total * p.H;
@@ -811,6 +872,11 @@ cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream
 cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream) {
   if (p.D == 64) return launch_d<64>(p, stream);
   if (p.D == 128) return launch_d<128>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwd_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream) {
+  if (p.D == 128) return launch_fp8_d128(p, f, stream);
   return cudaErrorInvalidValue;
 }
 

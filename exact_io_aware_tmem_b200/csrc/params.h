@@ -113,6 +113,14 @@ struct DecodeArgs {
   float* lse_part;           // [n_split, B*q_len, H] fp32 (n_split > 1)
 };
 
+// E4M3 forward: per-block steps of the quantised Q and K (pass 1 output),
+// [B, H, n_blocks] and [B, H_kv, n_blocks] fp32, n_blocks = ceil(N / 128).
+struct Fp8Args {
+  const float* q_scale;
+  const float* k_scale;
+  int n_blocks;
+};
+
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const AttnParams& p, cudaStream_t stream);
@@ -120,6 +128,11 @@ cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream);
 // mask: bit 0 preprocess (D_i), bit 1 dK/dV kernel, bit 2 dQ kernel.
 cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned mask);
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
+// E4M3 forward (D = 128) on codes from launch_fp8_quantize.
+cudaError_t launch_fwd_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream);
+// Pass 1: bf16 x [B*N, Hx, D] -> E4M3 codes x8 and per-block steps [B, Hx, nb].
+cudaError_t launch_fp8_quantize(const void* x, void* x8, float* scale, int B, int N, int Hx,
+                                int D, cudaStream_t stream);
 // Decode partials (and the combine kernel when d.n_split > 1).
 cudaError_t launch_decode_bf16(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream);
 
@@ -128,6 +141,10 @@ cudaError_t launch_decode_bf16(const AttnParams& p, const DecodeArgs& d, cudaStr
 // box of box_cols x box_rows and 128-byte swizzle. Returns false on failure.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long rows,
                        unsigned long long cols, unsigned box_cols, unsigned box_rows);
+
+// Host: as make_tmap_bf16_2d for a byte tensor (E4M3 codes), cols in bytes.
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, unsigned long long rows,
+                     unsigned long long cols, unsigned box_cols, unsigned box_rows);
 
 // Host: 3-D bf16 view (D, heads, rows) of a token-major [rows, heads, D]
 // tensor with a (64, box_heads, box_rows) box and 128-byte swizzle. Column

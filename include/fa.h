@@ -294,6 +294,43 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, voi
                     int max_seqlen_k, int causal, float scale, int n_split, void* workspace,
                     size_t ws_bytes, fa_stream_t stream);
 
+/*
+ * ------------------------------------------------------------------ FP8 ---
+ * FP8 (E4M3) forward (aiqz.cc "Flash Attention V2/V3 optimization" article,
+ * section "FP8 low precision"): pass 1 (fa_fp8_quantize) takes each block's
+ * largest |x|, its step Delta = max|x| / 448, and stores round(x / Delta) as
+ * E4M3 codes; pass 2 (fa_fwd_fp8) multiplies the quantised Q and K on the
+ * tensor cores with an fp32 accumulator and otherwise runs the forward above
+ * (P V in bf16 with fp32 accumulation, bf16 O, fp32 LSE). A block is 128
+ * consecutive tokens of one head of one sequence (the last block of a
+ * sequence may be shorter); Delta and x / Delta are IEEE single-precision
+ * divisions; rounding is to nearest even with saturation at +-448; a block of
+ * zeros gets Delta = 1. Dense batches only (no cu_seqlens).
+ *
+ * fa_fp8_quantize - pass 1 for one tensor.
+ *   x      bf16 [B * N, Hx, D] (token-major, as q or k of fa_fwd)
+ *   x8     out: E4M3 codes, one byte per element, same layout as x
+ *   scale  out: fp32 [B, Hx, ceil(N / 128)] steps Delta
+ *   D      a multiple of 8, at most 256. Pointers 16-byte aligned.
+ */
+fa_status fa_fp8_quantize(const void* x, void* x8, float* scale, int B, int N, int Hx, int D,
+                          fa_stream_t stream);
+
+/*
+ * fa_fwd_fp8 - pass 2: causal or full attention on the quantised Q and K.
+ *   q8, k8     E4M3 codes [B * N, H, D] / [B * N, H_kv, D] from fa_fp8_quantize
+ *   v          bf16 [B * N, H_kv, D]
+ *   q_scale,   fp32 [B, H, ceil(N / 128)] / [B, H_kv, ceil(N / 128)] steps
+ *   k_scale
+ *   o, lse     as for fa_fwd with cu_seqlens NULL (o bf16 [B * N, H, D],
+ *              lse fp32 [B, H, N])
+ *   D          128 (one 128-byte E4M3 row per token). scale <= 0: 1 / sqrt(D).
+ * Errors as for fa_fwd.
+ */
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v, const float* q_scale,
+                     const float* k_scale, void* o, float* lse, int B, int H, int H_kv, int N,
+                     int D, int causal, float scale, fa_stream_t stream);
+
 /* fa_version - library version as major * 10000 + minor * 100 + patch. */
 int fa_version(void);
 

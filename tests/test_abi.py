@@ -158,3 +158,19 @@ def test_decode_split_count_and_workspace_size(lib):
         return (x + 255) // 256 * 256
     assert lib.fa_decode_workspace_size(2, 1, 8, 2, 128, 1000, 3) == r256(rows * 128 * 4) + \
         r256(rows * 4)
+
+
+# --------------------------------------------------------------------- FP8 ---
+
+def test_fp8_entry_points_reject_bad_shapes(lib):
+    assert lib.fa_fp8_quantize(None, None, None, 1, 10, 2, 12, None) == _abi.FA_ERR_UNSUPPORTED
+    assert lib.fa_fp8_quantize(None, None, None, 1, 10, 2, 512, None) == _abi.FA_ERR_UNSUPPORTED
+    assert lib.fa_fp8_quantize(None, None, None, 1, 10, 2, 128, None) == _abi.FA_ERR_INVALID_ARG
+    assert lib.fa_fp8_quantize(None, None, None, 0, 10, 2, 128, None) == _abi.FA_OK
+    f = lib.fa_fwd_fp8
+    assert f(None, None, None, None, None, None, None, 1, 4, 2, 64, 64, 1, -1.0, None) == \
+        _abi.FA_ERR_UNSUPPORTED   # D = 64: one 128-byte E4M3 row per token is required
+    assert f(None, None, None, None, None, None, None, 1, 4, 3, 64, 128, 1, -1.0, None) == \
+        _abi.FA_ERR_INVALID_ARG   # H % H_kv != 0
+    assert f(None, None, None, None, None, None, None, 1, 4, 2, 64, 128, 1, -1.0, None) == \
+        _abi.FA_ERR_INVALID_ARG   # null tensors

@@ -1,0 +1,95 @@
+"""GPU parity of the FP8 (E4M3) forward against the float64 oracle (oracle/fp8.py).
+
+Pass 1 (fa_fp8_quantize) takes integer decisions - which E4M3 code each
+element gets - in single precision on both sides, so its codes and steps must
+match the oracle's exactly. Pass 2 (fa_fwd_fp8) is checked against attention on
+the dequantised inputs with the forward's bf16 bounds: |O - O_ref| <= 1.5e-2 +
+2^-9 |O_ref| and max-abs 1e-3 on LSE.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_tmem_b200 as fa
+from exact_io_aware_tmem_b200.workloads import WORKLOADS, make_inputs, random_case
+from oracle import attention as oa
+from oracle import fp8 as of
+from tests._util import f64, max_abs, o_excess_bf16
+
+pytestmark = pytest.mark.gpu
+
+O_TOL = 1.5e-2
+LSE_TOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from exact_io_aware_tmem_b200 import build
+    build.build()
+
+
+def _codes_as_values(x8: torch.Tensor) -> np.ndarray:
+    return x8.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("B,N,Hx,D", [(2, 300, 3, 128), (1, 128, 2, 64), (3, 1, 1, 128),
+                                      (1, 1000, 4, 8)])
+def test_quantize_codes_and_steps_are_exact(B, N, Hx, D):
+    inp = random_case(7 + N, dtype="bf16", lengths=[N] * B, H=Hx, H_kv=Hx, D=D, varlen=False,
+                      std=3.0)
+    x = inp.q
+    x[: min(N, 128)] = 0.0          # an all-zero first block (Delta = 1)
+    x8, sc = fa.fp8_quantize(x.cuda(), B, N)
+    torch.cuda.synchronize()
+    xh, d = of.quantize_blocks(x, B, N)
+    np.testing.assert_array_equal(sc.cpu().numpy(), d)
+    np.testing.assert_array_equal(_codes_as_values(x8), xh)
+
+
+def _fp8_case(inp, B, N, causal, scale):
+    q8, qs = fa.fp8_quantize(inp.q.cuda(), B, N)
+    k8, ks = fa.fp8_quantize(inp.k.cuda(), B, N)
+    o, lse = fa.fwd_fp8(q8, k8, inp.v.cuda(), qs, ks, B=B, N=N, causal=causal, scale=scale)
+    st, where = fa.check_device_error()
+    assert st == 0, f"device error {st} at {where:#x}"
+    return f64(o), f64(lse)
+
+
+def _check(o, lse, o_ref, lse_ref):
+    assert np.isfinite(o).all()
+    excess = o_excess_bf16(o, o_ref, O_TOL)
+    assert excess <= 0, f"O outside the bf16 bound by {excess} (max-abs {max_abs(o, o_ref)})"
+    err = max_abs(lse, lse_ref)
+    assert err <= LSE_TOL, f"LSE max-abs {err}"
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,N,H,H_kv", [(2, 300, 4, 2), (1, 129, 2, 1), (1, 1024, 8, 8)])
+def test_fp8_forward_small(B, N, H, H_kv, causal):
+    inp = random_case(11 + N, dtype="bf16", lengths=[N] * B, H=H, H_kv=H_kv, D=128, varlen=False,
+                      std=2.0)
+    scale = 128 ** -0.5
+    o, lse = _fp8_case(inp, B, N, causal, scale)
+    o_ref, lse_ref = of.fp8_forward(inp.q, inp.k, inp.v, B, N, causal, scale)
+    _check(o.reshape(B * N, H, 128), lse, o_ref, oa.lse_dense_layout(lse_ref, B, N))
+
+
+@pytest.mark.slow
+def test_fp8_forward_full_workload_sampled():
+    # The causal B2 H16 N8192 D128 inputs (Q, K x 2.0) through both passes; the
+    # oracle dequantises Q and K in full and forms sampled rows.
+    w = WORKLOADS["bf16_causal_b2_h16_n8192_d128"]
+    inp = make_inputs(w)
+    B, N, H = w.B, w.N, w.H
+    o, lse = _fp8_case(inp, B, N, True, w.scale)
+    o = o.reshape(B * N, H, w.D)
+    qh, dq = of.quantize_blocks(inp.q, B, N)
+    kh, dk = of.quantize_blocks(inp.k, B, N)
+    qd, kd = of.dequantize(qh, dq, B, N), of.dequantize(kh, dk, B, N)
+    v = inp.v.double().numpy()
+    rows = np.array([0, 1, 127, 128, 4095, 5000, 8190, 8191])
+    for b in range(B):
+        for h in (0, 7, 15):
+            sl = slice(b * N, (b + 1) * N)
+            o_ref, lse_ref = oa.head_forward(qd[sl, h], kd[sl, h], v[sl, h], w.scale, True, rows)
+            _check(o[b * N + rows, h], lse[b, h, rows], o_ref, lse_ref)
