@@ -14,6 +14,10 @@ path instead: a step is one fa_decode call (split partials + merge) of the
 q_len newest tokens of every sequence against its KV cache, resident in HBM;
 the metric is the KV-cache bytes it must read per second.
 
+``--workload fp8_fwd_causal_b2_h16_n8192_d128`` times the FP8 (E4M3)
+forward on that workload's inputs: a step is pass 1 (fa_fp8_quantize of Q and
+of K) plus pass 2 (fa_fwd_fp8); the metric is forward TFLOP/s.
+
 With N > 1 (launched by torch.distributed.run) every rank runs its own
 independently seeded batch of the same shape (the (batch, head) units are
 independent; no collective on the data path): weak scaling, timed as the
@@ -40,6 +44,9 @@ METRIC = "attention fwd/bwd TFLOP/s (bf16, device-timed) and % of B200 dense BF1
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "bf16_causal_b2_h16_n8192_d128"
 L2_BYTES = 126 * 1024 * 1024
+FP8_METRIC = "attention forward TFLOP/s, FP8 E4M3 Q K^T (two-pass, device-timed)"
+# FP8 workloads run the two passes on the inputs of the named bf16 workload.
+FP8_WORKLOADS = {"fp8_fwd_causal_b2_h16_n8192_d128": "bf16_causal_b2_h16_n8192_d128"}
 DECODE_METRIC = "split-KV decode attention, KV-cache GB/s read (bf16, device-timed)"
 DECODE_UNIT = "GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -97,7 +104,8 @@ def source_sha(*names) -> str:
 KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
-                  "decode": ("fwd_bf16.cu", "common.cuh", "params.h")}
+                  "decode": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "fp8_fwd": ("fwd_bf16.cu", "common.cuh", "params.h")}
 
 
 def recorded_traffic(kernel: str, workload: str):
@@ -427,6 +435,188 @@ def run_ours(args, w) -> None:
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- FP8 arm ---
+
+def fp8_oracle_sample(w, n_tokens: int):
+    """Pass 1 + pass 2 of the FP8 forward with the float64 oracle on one head
+    of the workload truncated to ``n_tokens``. Returns (seconds, FLOPs)."""
+    from exact_io_aware_tmem_b200.workloads import random_case
+    from oracle import fp8 as of
+    inp = random_case(w.seed, dtype=w.dtype, lengths=[n_tokens], H=1, H_kv=1, D=w.D, varlen=False,
+                      std=w.qk_mult)
+    t0 = time.perf_counter()
+    of.fp8_forward(inp.q, inp.k, inp.v, 1, n_tokens, w.causal, w.scale)
+    dt = time.perf_counter() - t0
+    fwd, _ = step_flops([n_tokens], 1, w.D, w.causal)
+    return dt, fwd
+
+
+def fp8_cpu_baseline(w, seconds: float) -> dict:
+    n = 512
+    t0, _ = fp8_oracle_sample(w, n)
+    n = max(128, min(w.N, int(n * math.sqrt(max(seconds, 0.05) / max(t0, 1e-3))) // 128 * 128))
+    dt, fl = fp8_oracle_sample(w, n)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "seconds": round(dt, 3),
+            "sample": f"float64 numpy FP8 oracle (block quantisation + attention on the "
+                      f"dequantised Q, K), one head of {w.name} truncated to N={n}"}
+
+
+def run_fp8_reference(args, name, w) -> None:
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    n = 1024
+    for _ in range(args.warmup):
+        fp8_oracle_sample(w, n)
+    tot_t = tot_f = 0.0
+    for _ in range(args.steps):
+        dt, fl = fp8_oracle_sample(w, n)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = f"float64 numpy FP8 oracle, one head of {w.name} truncated to N={n} per step"
+    line = {"impl": "reference", "metric": FP8_METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(config_of(w), **{"workload": name, "pass": "fp8 fwd"}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_fp8(args, name, w) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import exact_io_aware_tmem_b200 as fa
+    from exact_io_aware_tmem_b200.workloads import Workload, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    peaks = load_peaks()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = fp8_cpu_baseline(w, args.cpu_seconds)
+    wr = Workload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})
+    inp = make_inputs(wr)
+    B, N = w.B, w.N
+    fwd_fl, _ = step_flops([N] * B, w.H, w.D, w.causal)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    q8, qs = fa.fp8_quantize(q, B, N)
+    k8, ks = fa.fp8_quantize(k, B, N)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, w.H, N), device=dev, dtype=torch.float32)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        fa.fp8_quantize(q, B, N, out=q8, scale=qs)
+        fa.fp8_quantize(k, B, N, out=k8, scale=ks)
+        if ev is not None:
+            ev[1].record()
+        fa.fwd_fp8(q8, k8, v, qs, ks, B=B, N=N, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        if ev is not None:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    st, where = fa.check_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where:#x} during warm-up")
+    gpu_uuid = ""
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        gpu_uuid = gpu_uuid if gpu_uuid.startswith("GPU-") else "GPU-" + gpu_uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_uuid)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    start.record()
+    for i in range(args.steps):
+        step(evs[i])
+    end.record()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    st, where = fa.check_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error {st} at {where:#x} in the timed region")
+    max_ms = reduce_max(start.elapsed_time(end), dev)
+    q_ms = reduce_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs), dev)
+    f_ms = reduce_max(statistics.mean(e[1].elapsed_time(e[2]) for e in evs), dev)
+    # End to end: bf16 Q, K, V in from pinned host memory, O and LSE out.
+    e2e_steps = max(3, min(args.steps, 20))
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = o.numel() * o.element_size() + lse.numel() * 4
+    torch.cuda.synchronize(dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record()
+    for _ in range(e2e_steps):
+        for dst, src in zip((q, k, v), (hq, hk, hv)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+    e_end.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e_start.elapsed_time(e_end), dev)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    value = aggregate(fwd_fl * args.steps, world, [max_ms / 1e3]) / 1e12
+    # Pass 2's two products: Q K^T at the E4M3 rate (twice bf16, the nominal
+    # ratio) and P V in bf16, half of the FLOPs each, so its tensor-core floor
+    # is 0.75 of the bf16 time: peak = measured sustained bf16 / 0.75.
+    peak = peaks["bf16_tflops_sustained"] / 0.75
+    achieved = fwd_fl / (f_ms / 1e3) / 1e12
+    line = {
+        "metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 Q K^T, bf16 P V",
+        "data": "synthetic",
+        "config": dict(config_of(w), **{"workload": name, "base_workload": w.name,
+                                         "pass": "fp8 fwd (quantise Q, K + forward)"},
+                       parallelism=f"replicas{world}" if world > 1 else "none",
+                       l2="not flushed: every step reads and writes > 200 MiB > 126 MiB L2",
+                       ranks="each rank its own seeded batch of this shape"),
+        "kernel_ms": {"fp8_quantize_kernel (Q and K)": round(q_ms, 4),
+                      "fwd_bf16_kernel<128, false, true>": round(f_ms, 4)},
+        "roofline": {"kernel": "fwd_bf16_kernel<128, false, true>", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "peak_kind": f"{peaks['source']} sustained bf16 / 0.75 (E4M3 Q K^T at the "
+                                  f"nominal 2x rate, bf16 P V)",
+                     "traffic": recorded_traffic("fp8_fwd", name)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": fwd_fl * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------- decode arm ---
 
 def decode_config(w) -> dict:
@@ -637,6 +827,13 @@ def main(argv=None) -> int:
     from exact_io_aware_tmem_b200.workloads import DECODE_WORKLOADS, WORKLOADS
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in FP8_WORKLOADS:
+        w = WORKLOADS[FP8_WORKLOADS[args.workload]]
+        if args.impl == "reference":
+            run_fp8_reference(args, args.workload, w)
+        else:
+            run_fp8(args, args.workload, w)
+        return 0
     if args.workload in DECODE_WORKLOADS:
         w = DECODE_WORKLOADS[args.workload]
         if args.impl == "reference":

@@ -153,12 +153,14 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     return out, lse
 
 
-def fp8_quantize(x: torch.Tensor, B: int, N: int):
+def fp8_quantize(x: torch.Tensor, B: int, N: int, *, out: Optional[torch.Tensor] = None,
+                 scale: Optional[torch.Tensor] = None):
     """Pass 1 of the FP8 forward: E4M3 codes (uint8, x's shape) and per-block
     steps fp32 [B, Hx, ceil(N / 128)] of a bf16 [B*N, Hx, D] (or [B, N, Hx, D]) tensor."""
     Hx, D = x.shape[-2], x.shape[-1]
-    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
-    sc = torch.empty((B, Hx, (N + 127) // 128), dtype=torch.float32, device=x.device)
+    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if out is None else out
+    sc = torch.empty((B, Hx, (N + 127) // 128), dtype=torch.float32, device=x.device) \
+        if scale is None else scale
     st = _abi.lib().fa_fp8_quantize(_ptr(x), _ptr(x8), _ptr(sc), B, N, Hx, D, _stream(x.device))
     _abi.check(st, "fa_fp8_quantize")
     return x8, sc
