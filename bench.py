@@ -627,14 +627,22 @@ def decode_config(w) -> dict:
             "cache_tokens": int(sum(lengths)), "pass": "decode", "seed": w.seed}
 
 
-def decode_oracle_sample(w, n_seq: int):
+def decode_oracle_case(w, n_seq: int):
+    """Seeded inputs of the first ``n_seq`` sequences of a decode workload."""
+    from exact_io_aware_tmem_b200.workloads import decode_case
+    return decode_case(w.seed, dtype=w.dtype, lengths=w.lengths()[:n_seq], q_len=w.q_len,
+                       H=w.H, H_kv=w.H_kv, D=w.D, page_size=w.page_size)
+
+
+def decode_oracle_sample(w, n_seq: int, c=None):
     """The float64 decode oracle on the first ``n_seq`` sequences of the
-    workload. Returns (seconds, KV bytes, FLOPs)."""
-    from exact_io_aware_tmem_b200.workloads import decode_bytes, decode_case, decode_flops
+    workload (``c``: their inputs, drawn if not given). Returns (seconds, KV
+    bytes, FLOPs)."""
+    from exact_io_aware_tmem_b200.workloads import decode_bytes, decode_flops
     from oracle import decode as od
     lengths = w.lengths()[:n_seq]
-    c = decode_case(w.seed, dtype=w.dtype, lengths=lengths, q_len=w.q_len, H=w.H, H_kv=w.H_kv,
-                    D=w.D, page_size=w.page_size)
+    if c is None:
+        c = decode_oracle_case(w, n_seq)
     t0 = time.perf_counter()
     od.decode_forward(c.q, c.k_cache, c.v_cache, c.cache_seqlens, q_len=w.q_len, scale=w.scale,
                       causal=w.causal, stride=c.page_size, page_size=c.page_size,
@@ -655,12 +663,18 @@ def decode_cpu_baseline(w) -> dict:
 def run_decode_reference(args, w) -> None:
     if int(os.environ.get("RANK", "0")) != 0:
         return
-    n = max(1, w.B // 4)
+    # About 150 s of oracle work over all steps: the sample is drawn once and
+    # is as many leading sequences as fit one step's share.
+    per_step = max(0.2, 150.0 / max(1, args.steps + args.warmup))
+    c1 = decode_oracle_case(w, 1)
+    t1, _, _ = decode_oracle_sample(w, 1, c1)
+    n = max(1, min(w.B, int(per_step / max(t1, 1e-3))))
+    c = c1 if n == 1 else decode_oracle_case(w, n)
     for _ in range(args.warmup):
-        decode_oracle_sample(w, n)
+        decode_oracle_sample(w, n, c)
     tot_t = tot_b = 0.0
     for _ in range(args.steps):
-        dt, by, _ = decode_oracle_sample(w, n)
+        dt, by, _ = decode_oracle_sample(w, n, c)
         tot_t += dt
         tot_b += by
     value = tot_b / tot_t / 1e9
