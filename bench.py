@@ -94,10 +94,17 @@ def reduce_max(value: float, device=None) -> float:
 
 
 def source_sha(*names) -> str:
+    """Hash of the code in the named csrc files: ``//`` comments and blank
+    lines are left out, so editing a comment does not orphan a capture."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "exact_io_aware_tmem_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "exact_io_aware_tmem_b200", "csrc", n)) as f:
+            for line in f:
+                if line.lstrip().startswith("//"):
+                    continue
+                code = line.split("//", 1)[0].rstrip() if '"' not in line else line.rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -13,16 +13,18 @@
 // recurrence up to rounding.
 //
 // How, on B200 (one CTA per 128-row Q tile, 320 threads):
-//   warp 8      TMA producer: Q tile once, then K_j and V_j tiles through
-//               separate multi-stage shared-memory rings (mbarrier full/empty
-//               pairs, 128-byte swizzle, no multicast);
-//   warp 9      MMA issuer (one thread): S_j = Q K_j^T with tcgen05.mma into
-//               TMEM score buffer j mod 2 (Q is the A operand, held in TMEM,
-//               so each tile streams only K and V through shared memory and
-//               the tensor core is not held back by shared-memory bandwidth),
-//               and O += P_j V_j with P read straight from its own TMEM
-//               columns as packed bf16. S_{j+2} is issued as soon as the
-//               softmax has loaded S_j, ahead of PV_j;
+//   warp 8      TMA producer (the whole warp runs its loop, lane 0 issues):
+//               the Q tile once, then K_j and V_j tiles through separate
+//               multi-stage shared-memory rings (mbarrier full/empty pairs,
+//               128-byte swizzle, no multicast), K loaded ahead of V whenever
+//               both rings have room;
+//   warp 9      MMA warp, converged, one elect.sync lane issuing: S_j =
+//               Q K_j^T with tcgen05.mma into TMEM score buffer j mod 2 (Q is
+//               the A operand, held in TMEM, so each tile streams only K and
+//               V through shared memory and the tensor core is not held back
+//               by shared-memory bandwidth), and O += P_j V_j with P read
+//               straight from its own TMEM columns as packed bf16. S_{j+2} is
+//               issued as soon as the softmax has loaded S_j, ahead of PV_j;
 //   warps 0-7   softmax, two groups of four warps; group g takes the key
 //               tiles j = g, g+2, g+4, ... One thread per query row (TMEM
 //               lane = row): it loads its 128 scores with tcgen05.ld,
@@ -31,6 +33,11 @@
 //               in TMEM when the reference max moved. Group 0 first copies Q
 //               from the swizzled shared tile into TMEM. At the end both
 //               groups merge their row sums and each writes half of O / l.
+// The same pipeline has two more instantiations (template flags, below):
+// split-KV decode over a contiguous or paged KV cache (agentalpha.top
+// "flash attention" answer, follow-up 2) and the FP8 (E4M3) forward, whose
+// score MMA reads E4M3 Q and K from shared memory (aiqz.cc article, section
+// "FP8 low precision").
 // The two groups run the same recurrence with one shared reference max per
 // row: the group on tile j takes the reference of tile j-1 from the other
 // group (a shared-memory word per row, published by an mbarrier arrive as
