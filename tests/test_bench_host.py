@@ -114,3 +114,34 @@ def test_warmup_below_three_rejected():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"],
                          capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    import bench
+    csrc = tmp_path / "exact_io_aware_tmem_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("// header\nint a = 1;  // trailing\n\nint b = 2;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.source_sha("k.cu")
+    (csrc / "k.cu").write_text("// a different header\n// more\nint a = 1;  // other words\nint b = 2;\n")
+    assert bench.source_sha("k.cu") == h0
+    (csrc / "k.cu").write_text("// header\nint a = 1;\nint b = 3;\n")
+    assert bench.source_sha("k.cu") != h0
+    # a quoted "//" inside code is code
+    (csrc / "k.cu").write_text('// header\nconst char* s = "a//b";\nint b = 2;\n')
+    h1 = bench.source_sha("k.cu")
+    (csrc / "k.cu").write_text('// header\nconst char* s = "a//c";\nint b = 2;\n')
+    assert bench.source_sha("k.cu") != h1
+
+
+def test_decode_bytes_and_flops_formulas():
+    from exact_io_aware_tmem_b200.workloads import (DECODE_WORKLOADS, decode_bytes,
+                                                    decode_flops)
+    # K and V, every cached token of every kv head, bf16
+    assert decode_bytes([10, 6], 2, 64) == 2 * 16 * 2 * 64 * 2
+    # two products of 2 * D flops per (query row, key)
+    assert decode_flops([10, 6], 3, 4, 64) == 4.0 * 3 * 4 * 64 * 16
+    w = DECODE_WORKLOADS["bf16_decode_b16_h32_kv8_d128_q1"]
+    L = w.lengths()
+    assert len(L) == 16 and min(L) >= 4096 and max(L) <= 32768
+    assert L == w.lengths()       # seeded
