@@ -273,6 +273,55 @@ def config_of(w) -> dict:
 
 # -------------------------------------------------------------- GPU arm ---
 
+def pipelined_e2e(torch, dev, host_in, dev_in, dev_out, run_step, steps: int) -> float:
+    """End-to-end device time (ms) of ``steps`` steps through the public API.
+
+    Every step copies its inputs host -> device from pinned memory, runs, and
+    reads its outputs back into pinned memory; all of it inside the timed
+    region. The copies of neighbouring steps overlap the computation, as a
+    serving or training loop would arrange: two sets of device buffers, one
+    stream per direction plus the compute stream, and events so that a
+    buffer set is refilled only after the step two back has finished with it
+    (inputs) and been read out (outputs).
+    """
+    sets_in = [dev_in, [torch.empty_like(t) for t in dev_in]]
+    sets_out = [dev_out, [torch.empty_like(t) for t in dev_out]]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in dev_out]
+                for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    e_in, e_cmp, e_out = ([ev() for _ in range(steps)] for _ in range(3))
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    start.record()
+    for st_ in (s_in, s_cmp, s_out):
+        st_.wait_event(start)
+    for i in range(steps):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(e_cmp[i - 2])      # step i-2 no longer reads set b
+            for dst, src in zip(sets_in[b], host_in):
+                dst.copy_(src, non_blocking=True)
+            e_in[i].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(e_in[i])
+            if i >= 2:
+                s_cmp.wait_event(e_out[i - 2])     # step i-2's outputs have been read out
+            run_step(sets_in[b], sets_out[b])
+            e_cmp[i].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(e_cmp[i])
+            for dst, src in zip(host_out[b], sets_out[b]):
+                dst.copy_(src, non_blocking=True)
+            e_out[i].record(s_out)
+    cur = torch.cuda.current_stream(dev)
+    for e in (e_in[-1], e_cmp[-1], e_out[-1]):
+        cur.wait_event(e)
+    end.record()
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(end)
+
 def run_ours(args, w) -> None:
     import torch
     import torch.distributed as dist
@@ -372,26 +421,22 @@ def run_ours(args, w) -> None:
     k_ms = {n: reduce_max(t, dev) for n, t in k_ms.items()}
 
     # End to end through the public API with host buffers: pinned H2D of the
-    # step's inputs, forward + backward, D2H of every output.
+    # step's inputs, forward + backward, D2H of every output, pipelined.
     e2e_steps = max(3, min(args.steps, 20))
-    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-    outs = (o, lse, dq, dk, dv)
-    houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    host_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
+    outs = [o, lse, dq, dk, dv]
     bytes_out = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step(ins, outs_):
+        qq, kk, vv, dd = ins
+        oo, ll, gq, gk, gv = outs_
+        fa.fwd(qq, kk, vv, out=oo, lse=ll, **kw)
+        fa.bwd(dd, qq, kk, vv, oo, ll, workspace=ws, dq=gq, dk=gk, dv=gv, **kw)
+
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize(dev)
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record()
-    for _ in range(e2e_steps):
-        for dst, src in zip((q, k, v, do), (hq, hk, hv, hdo)):
-            dst.copy_(src, non_blocking=True)
-        step()
-        for dst, src in zip(houts, outs):
-            dst.copy_(src, non_blocking=True)
-    e_end.record()
-    torch.cuda.synchronize(dev)
-    e2e_ms = reduce_max(e_start.elapsed_time(e_end), dev)
+    e2e_ms = reduce_max(pipelined_e2e(torch, dev, host_in, [q, k, v, do], outs, e2e_step,
+                                      e2e_steps), dev)
 
     if world > 1:
         dist.barrier()
@@ -435,7 +480,9 @@ def run_ours(args, w) -> None:
         "cpu_baseline": cpu,
         "e2e": {"value": per_step_fl * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "steps": e2e_steps, "h2d_bytes_per_step": bytes_in,
-                "d2h_bytes_per_step": bytes_out},
+                "d2h_bytes_per_step": bytes_out,
+                "how": "public API, pinned host buffers, copies of neighbouring steps "
+                       "overlapping the computation (double-buffered, three streams)"},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
@@ -567,25 +614,23 @@ def run_fp8(args, name, w) -> None:
     max_ms = reduce_max(start.elapsed_time(end), dev)
     q_ms = reduce_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs), dev)
     f_ms = reduce_max(statistics.mean(e[1].elapsed_time(e[2]) for e in evs), dev)
-    # End to end: bf16 Q, K, V in from pinned host memory, O and LSE out.
+    # End to end: bf16 Q, K, V in from pinned host memory, both passes, O and
+    # LSE out, pipelined.
     e2e_steps = max(3, min(args.steps, 20))
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = o.numel() * o.element_size() + lse.numel() * 4
-    torch.cuda.synchronize(dev)
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record()
-    for _ in range(e2e_steps):
-        for dst, src in zip((q, k, v), (hq, hk, hv)):
-            dst.copy_(src, non_blocking=True)
-        step()
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
-    e_end.record()
-    torch.cuda.synchronize(dev)
-    e2e_ms = reduce_max(e_start.elapsed_time(e_end), dev)
+
+    def e2e_step(ins, outs_):
+        qq, kk, vv = ins
+        oo, ll = outs_
+        fa.fp8_quantize(qq, B, N, out=q8, scale=qs)
+        fa.fp8_quantize(kk, B, N, out=k8, scale=ks)
+        fa.fwd_fp8(q8, k8, vv, qs, ks, B=B, N=N, causal=w.causal, scale=w.scale, out=oo, lse=ll)
+
+    if world > 1:
+        dist.barrier()
+    e2e_ms = reduce_max(pipelined_e2e(torch, dev, [t.cpu().pin_memory() for t in (q, k, v)],
+                                      [q, k, v], [o, lse], e2e_step, e2e_steps), dev)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -617,7 +662,9 @@ def run_fp8(args, name, w) -> None:
                      "traffic": recorded_traffic("fp8_fwd", name)},
         "cpu_baseline": cpu,
         "e2e": {"value": fwd_fl * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
-                "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "public API, pinned host buffers, copies of neighbouring steps "
+                       "overlapping the computation (double-buffered, three streams)"},
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }
