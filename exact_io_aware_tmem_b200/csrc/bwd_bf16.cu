@@ -20,19 +20,24 @@
 //                      dV  += P^T dO_i,  dK += dS^T Q_i (A operands from TMEM)
 //   bwd_dq           one CTA per (sequence, query head, 128-row query tile);
 //                    Q and dO stay in shared memory while K_j, V_j stream
-//                    through a ring. Queries on the TMEM lanes:
-//                      S = Q K_j^T (double-buffered), dP = dO V_j^T
+//                    through their own rings. Queries on the TMEM lanes:
+//                      S = Q K_j^T (one buffer, handed back as soon as its
+//                      softmax group has loaded it), dP = dO V_j^T (one
+//                      buffer per group)
 //                      dS = P * (dP - D) -> bf16 over dP,  dQ += dS K_j
 //                    then dQ = bf16(scale dQ), each row written once.
 // Recomputing S and dP in bwd_dq costs two extra products per tile pair, and
 // buys what the single fused kernel could not have at once on this part: only
-// 128-wide tensor-core instructions (64-wide ones run well below the 128-wide
-// rate), P and dS as TMEM operands (no dS round trip through shared memory),
-// no atomic dQ accumulation and no fp32 dQ workspace.
+// 128-wide tensor-core instructions (64-wide ones with both operands in shared
+// memory are bound by shared-memory bandwidth), P and dS as TMEM operands (no
+// dS round trip through shared memory), no atomic dQ accumulation and no fp32
+// dQ workspace.
 //
 // Roles in both kernels (320 threads): warps 0-7 softmax / dS (thread = TMEM
-// lane row; warps w and w+4 share a lane quarter and split the 128 columns in
-// halves), warp 8 TMA producer, warp 9 MMA issuer (one thread).
+// lane row; dK/dV: warps w and w+4 share a lane quarter and split the 128
+// columns in halves; dQ: two groups of four warps on alternate key tiles),
+// warp 8 TMA producer, warp 9 MMA warp (converged, one elect.sync lane
+// issuing the tensor-core instructions).
 // D = 64 runs the D = 128 code: the tensor maps are 3-D (D, heads, tokens), so
 // the second 64-wide column block is out of bounds and arrives as zeros.
 #include <limits.h>

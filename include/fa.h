@@ -7,7 +7,10 @@
  * exponential sum l, rescaling of the output accumulator, one division by l at
  * the end), and saves the row log-sum-exp for the backward pass. The backward
  * pass recomputes S and P from Q, K and the saved log-sum-exp and forms dV, dP,
- * dS, dQ and dK; no N x N matrix is ever written to global memory.
+ * dS, dQ and dK; no N x N matrix is ever written to global memory. Two more
+ * paths reuse the forward: split-KV decode over a contiguous or paged KV cache
+ * (fa_decode) and the two-pass FP8 (E4M3) forward (fa_fp8_quantize,
+ * fa_fwd_fp8); their sections below state their sources and conventions.
  *
  * Sources for what is computed:
  *   - aiqz.cc "Flash Attention V2/V3 optimization", section "IO bottleneck
@@ -48,7 +51,8 @@
  *   LSE_i = m_i + ln(l_i).
  * Pointers: device pointers, 16-byte aligned (tensor-memory-accelerator
  *   copies need it). Buffers are owned by the caller; the library allocates
- *   no device memory and keeps no per-call state.
+ *   no device memory and keeps no per-call state (fa_bwd_noalloc's built-in
+ *   scratch array is part of the loaded library, see its section).
  * Streams: every entry point only enqueues work on ``stream`` (NULL = the
  *   legacy default stream) and returns without synchronising, except
  *   fa_check_device_error.
