@@ -12,7 +12,8 @@
 // in base 2 on pre-scaled logits (scale * log2 e), which is the same
 // recurrence up to rounding.
 //
-// How, on B200 (one CTA per 128-row Q tile, 320 threads):
+// How, on B200 (one CTA per 128-row Q tile; 352 threads at D = 128, 320 at
+// D = 64):
 //   warp 8      TMA producer (the whole warp runs its loop, lane 0 issues):
 //               the Q tile once, then K_j and V_j tiles through separate
 //               multi-stage shared-memory rings (mbarrier full/empty pairs,
@@ -22,9 +23,11 @@
 //               Q K_j^T with tcgen05.mma into TMEM score buffer j mod 2 (Q is
 //               the A operand, held in TMEM, so each tile streams only K and
 //               V through shared memory and the tensor core is not held back
-//               by shared-memory bandwidth), and O += P_j V_j with P read
-//               straight from its own TMEM columns as packed bf16. S_{j+2} is
-//               issued as soon as the softmax has loaded S_j, ahead of PV_j;
+//               by shared-memory bandwidth) as soon as the softmax has loaded
+//               S_{j-2};
+//   warp 10     (D = 128) the same for O += P_j V_j, with P read straight
+//               from its own TMEM columns as packed bf16. At D = 64 warp 9
+//               issues these too, QK_{j+2} ahead of each PV_j;
 //   warps 0-7   softmax, two groups of four warps; group g takes the key
 //               tiles j = g, g+2, g+4, ... One thread per query row (TMEM
 //               lane = row): it loads its 128 scores with tcgen05.ld,
@@ -59,8 +62,8 @@ namespace {
 constexpr int BM = 128;  // query rows per CTA (= TMEM lanes)
 constexpr int BN = 128;  // keys per tile
 constexpr int WARP_TMA = 8;
-constexpr int WARP_MMA = 9;
-constexpr int THREADS = 320;
+constexpr int WARP_MMA = 9;   // MMA issuer (and the TMEM allocation)
+constexpr int WARP_PV = 10;   // P V issuer when the MMAs are split over two warps
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S0 = 0;
 constexpr uint32_t TM_O = 256;
@@ -86,6 +89,12 @@ template <int D, bool F8>
 struct FwdCfg {
   static_assert(!F8 || D == 128, "the E4M3 path has one 128-byte row per token");
   static constexpr int STAGES = (D == 64 || F8) ? 4 : 3;
+  // D = 128: one warp issues the score MMAs and another the P V MMAs, so a
+  // score MMA never waits behind the P V product of the tile before it.
+  // D = 64 (half the MMA work per exponential): one warp issues both in a
+  // fixed interleave, measured faster there.
+  static constexpr bool SPLIT_MMA = D == 128;
+  static constexpr int THREADS = SPLIT_MMA ? 352 : 320;
   static constexpr int CHUNKS = D / 64;            // 128-byte blocks of a bf16 row
   static constexpr int QK_CHUNKS = F8 ? 1 : CHUNKS; // 128-byte blocks of a Q / K row
   static constexpr uint32_t TILE = BM * D * 2;     // bytes of one bf16 128-row tile
@@ -149,7 +158,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
 // block (pass 1, fp8.cu); S = Q_hat K_hat^T runs as a kind::f8f6f4 MMA with
 // fp32 accumulation and is scaled by Delta_Q Delta_K of its two blocks.
 template <int D, bool DEC, bool F8>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m,
@@ -440,27 +449,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(bars.v_empty(st), ph, p.err, abort, W_VEMPTY)) break;
       }
     }
-  } else if (warp == WARP_MMA) {
-    // -------------------------------------------------------- MMA issuer ---
+  } else if (warp == WARP_MMA || (C::SPLIT_MMA && warp == WARP_PV)) {
+    // -------------------------------------------------------- MMA issuers ---
     // The whole warp runs the loop (waits and operands stay warp-uniform);
-    // one elected lane issues the tensor-core instructions and commits.
+    // one elected lane issues the tensor-core instructions and commits. A
+    // commit tracks the tcgen05 operations its own thread issued.
+    //   S_j = Q K_j^T into score buffer j mod 2 (M=128, N=128, K=D in steps
+    //   of 16) once K_j has landed and the buffer's group has loaded S_{j-2};
+    //   O += P_j V_j (M=128, N=D, K=128 keys in steps of 16) once V_j has
+    //   landed and P_j is in TMEM. One thread issues every P V product, so
+    //   they run in key order on the single O accumulator.
+    // Split (two warps): the score warp runs up to two tiles ahead on its
+    // own. Single warp: QK_0 and QK_1 first, then QK_{j+2} ahead of each PV_j.
+    const bool do_qk = warp == WARP_MMA;
+    const bool do_pv = !C::SPLIT_MMA || warp == WARP_PV;
     const uint32_t leader = elect_one();
     constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
+    constexpr uint32_t IDESC_QK8 = idesc_e4m3(BM, BN);
     constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
-    // Shared-memory descriptors, built once and stepped by constant offsets.
     const uint64_t k_desc = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
     const uint64_t q_desc = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);   // E4M3 path only
-    constexpr uint32_t IDESC_QK8 = idesc_e4m3(BM, BN);
     const uint64_t v_desc = sdesc_sw128(sbase + C::OFF_V, CHUNK_BYTES, 1024);
     // Q reaches TMEM through the softmax threads.
     bool ok = warp_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM);
     if (ok) tc_fence_after();
-    // S_j = Q K_j^T into score buffer j mod 2 (M=128, N=128, K=D in steps
-    // of 16) for j = jq; the buffer is free once its group has loaded
-    // S_{j-2}. QK_0 and QK_1 go first, then QK_{j+2} ahead of each PV_j.
-    int jq = 0;
+    int jq = do_qk ? 0 : n_kv;
     for (int j = -2; j < n_kv && ok; ++j) {
-      for (; jq < n_kv && jq <= j + 2; ++jq) {
+      const int jq_end = C::SPLIT_MMA ? n_kv : min(n_kv, j + 3);
+      for (; jq < jq_end; ++jq) {
         const int st = jq % C::STAGES;
         if (!warp_wait(bars.k_full(st), (jq / C::STAGES) & 1, p.err, abort, W_KFULL) ||
             (jq >= 2 &&
@@ -480,16 +496,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-            mma_ts_if(leader, d_s, tmem + TM_Q + kk * 8, sdesc_add(k_desc, st * C::QK_TILE + off),
-                      IDESC_QK, kk > 0);
+            mma_ts_if(leader, d_s, tmem + TM_Q + kk * 8,
+                      sdesc_add(k_desc, st * C::QK_TILE + off), IDESC_QK, kk > 0);
           }
         }
         tc_commit_if(leader, bars.s_full(jq & 1));
         tc_commit_if(leader, bars.k_empty(st));
       }
-      if (!ok) break;
+      if (!ok || !do_pv) break;
       if (j < 0) continue;
-      // O += P_j V_j: M=128, N=D, K=128 keys in steps of 16.
       const int st = j % C::STAGES;
       if (!warp_wait(bars.v_full(st), (j / C::STAGES) & 1, p.err, abort, W_VFULL)) break;
       if (v_tail && j == n_kv - 1 && !warp_wait(bars.v_fix(), 0, p.err, abort, W_VFIX)) break;
@@ -819,7 +834,7 @@ cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int group = l2_group(4ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_bf16_kernel<D, false, false><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
+  fwd_bf16_kernel<D, false, false><<<static_cast<unsigned>(tiles), C::THREADS, C::SMEM, stream>>>(
       tq, tk, tv, p, num_m, group, DecodeArgs{}, Fp8Args{});
   return cudaGetLastError();
 }
@@ -841,7 +856,7 @@ cudaError_t launch_fp8_d128(const AttnParams& p, const Fp8Args& f, cudaStream_t 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int group = l2_group(3ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_bf16_kernel<D, false, true><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
+  fwd_bf16_kernel<D, false, true><<<static_cast<unsigned>(tiles), C::THREADS, C::SMEM, stream>>>(
       tq, tk, tv, p, num_m, group, DecodeArgs{}, f);
   return cudaGetLastError();
 }
@@ -864,7 +879,7 @@ cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream
   cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, true, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  fwd_bf16_kernel<D, true, false><<<static_cast<unsigned>(ctas), THREADS, C::SMEM, stream>>>(
+  fwd_bf16_kernel<D, true, false><<<static_cast<unsigned>(ctas), C::THREADS, C::SMEM, stream>>>(
       tq, tk, tv, p, 0, 0, d, Fp8Args{});
   e = cudaGetLastError();
   if (e != cudaSuccess || d.n_split == 1) return e;
