@@ -132,15 +132,17 @@ constexpr uint32_t OFF_DO = OFF_Q + QS * TILE;
 constexpr uint32_t OFF_LSE = OFF_DO + QS * TILE;   // float [QS][BT]: LSE * log2(e)
 constexpr uint32_t OFF_DLT = OFF_LSE + QS * BT * 4;  // float [QS][BT]: D_i
 constexpr uint32_t OFF_BAR = OFF_DLT + QS * BT * 4;
-// kv_full, q_full[QS], q_empty[QS], s_full, dp_full, p_ready, ds_ready, dkv_done
-constexpr int NBAR = 1 + 2 * QS + 5;
+// kv_full, q_full[QS], q_empty[QS], s_full, dp_full, p_ready, ds_ready,
+// dkv_done, do_full[QS]. A stage's Q (with its LSE and D_i) and its dO land
+// on separate barriers, so S^T_t needs only Q_t.
+constexpr int NBAR = 1 + 3 * QS + 5;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(SMEM <= 232448, "shared memory budget");
 
 enum : unsigned {
   W_KV = 0x20100, W_QEMPTY = 0x20200, W_QFULL = 0x20300, W_SFULL = 0x20400, W_PREADY = 0x20500,
-  W_DPFULL = 0x20600, W_DSREADY = 0x20700, W_DKV = 0x20800
+  W_DPFULL = 0x20600, W_DSREADY = 0x20700, W_DKV = 0x20800, W_DOFULL = 0x20900
 };
 
 struct Bars {
@@ -153,6 +155,7 @@ struct Bars {
   __device__ uint32_t p_ready() const { return b + 8u * (3 + 2 * QS); }
   __device__ uint32_t ds_ready() const { return b + 8u * (4 + 2 * QS); }
   __device__ uint32_t dkv_done() const { return b + 8u * (5 + 2 * QS); }
+  __device__ uint32_t do_full(int s) const { return b + 8u * (6 + 2 * QS + s); }
 };
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -191,8 +194,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort = 0;
     mbar_init(bars.kv_full(), 1);
     for (int s = 0; s < QS; ++s) {
-      mbar_init(bars.q_full(s), 2);  // TMA bytes + staged LSE / D_i
+      mbar_init(bars.q_full(s), 2);  // Q bytes + staged LSE / D_i
       mbar_init(bars.q_empty(s), 1);
+      mbar_init(bars.do_full(s), 1);  // dO bytes
     }
     mbar_init(bars.s_full(), 1);
     mbar_init(bars.dp_full(), 1);
@@ -246,9 +250,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!warp_wait(bars.q_empty(st), ((t / QS) & 1) ^ 1, p.err, abort, W_QEMPTY)) break;
       if (lane == 0) {
         const int row_q = sq.start + qbase;
-        mbar_arrive_expect_tx(bars.q_full(st), 2 * TILE);
+        mbar_arrive_expect_tx(bars.q_full(st), TILE);
         load_tile(sbase + OFF_Q + st * TILE, &tm_q, bars.q_full(st), h, row_q);
-        load_tile(sbase + OFF_DO + st * TILE, &tm_do, bars.q_full(st), h, row_q);
+        mbar_arrive_expect_tx(bars.do_full(st), TILE);
+        load_tile(sbase + OFF_DO + st * TILE, &tm_do, bars.do_full(st), h, row_q);
       }
 #pragma unroll
       for (int k = 0; k < BT / 32; ++k) {
@@ -301,6 +306,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ok) {
           tc_fence_after();
           issue_s(0);
+        }
+        ok = ok && warp_wait(bars.do_full(0), 0, p.err, abort, W_DOFULL);
+        if (ok) {
+          tc_fence_after();
           issue_dp(0);
         }
       }
@@ -330,7 +339,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kk = 0; kk < BT / 16; ++kk)
           mma_ts_if(leader, tmem + TM_DK, tmem + TM_DP + packed_col(kk),
                  sdesc_add(q_mn, st * TILE + kk * 2048), ID_DVK, (t > 0 || kk > 0) ? 1u : 0u);
-        if (more) issue_dp(sn);
+        if (more) {
+          if (!(ok = warp_wait(bars.do_full(sn), ((t + 1) / QS) & 1, p.err, abort, W_DOFULL)))
+            break;
+          tc_fence_after();
+          issue_dp(sn);
+        }
         tc_commit_if(leader, bars.q_empty(st));
       }
       tc_commit_if(leader, bars.dkv_done());
