@@ -24,6 +24,12 @@ def test_dense_workloads_shapes_and_flops():
     w = WORKLOADS["bf16_fwd_b4_h16_n2048_d64"]
     fl_f, _ = flops([w.N] * w.B, w.H, w.D, w.causal)
     assert round(fl_f / 1e9, 1) == 68.7
+    w = WORKLOADS["bf16_gqa_causal_b1_h32_kv8_n16384_d128"]
+    fl_f, fl_b = flops([w.N] * w.B, w.H, w.D, w.causal)
+    assert round(fl_f / 1e9, 1) == 2199.0 and round(fl_b / 1e9, 1) == 5497.6
+    w = WORKLOADS["bf16_varlen_h16_d128_16seqs"]
+    fl_f, fl_b = flops(make_inputs(w).cu_seqlens.diff().tolist(), w.H, w.D, w.causal)
+    assert round(fl_f / 1e9, 1) == 685.3 and round(fl_b / 1e9, 1) == 1713.4
 
 
 def test_inputs_are_reproducible():
