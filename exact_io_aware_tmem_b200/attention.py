@@ -85,8 +85,8 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         dv: Optional[torch.Tensor] = None, phases: int = 7):
     """Attention backward for the loss sum(O * dO). Returns (dQ, dK, dV).
 
-    ``phases`` selects the kernels to enqueue (bit 0 preprocess, bit 1 main,
-    bit 2 dQ conversion); the default runs all three.
+    ``phases`` selects the kernels to enqueue (bit 0 the D_i preprocess, bit 1
+    the dK / dV kernel, bit 2 the dQ kernel); the default runs all three.
     """
     B, N, H, H_kv, D, max_sl, T = _shape(q, k, cu_seqlens, max_seqlen)
     for t in (dout, o, v, lse):

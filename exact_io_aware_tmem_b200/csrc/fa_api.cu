@@ -111,6 +111,18 @@ fa_status check_common(AttnParams& p, int B, int H, int H_kv, int N, int D, fa_d
 
 }  // namespace
 
+fa_status record_cuda(cudaError_t e) { return cuda_status(e); }
+
+fa_status check_bwd_sizes(int B, int H, int H_kv, int N, int D, fa_dtype dtype, int causal,
+                          const int* cu_seqlens, int max_seqlen, long long total_tokens,
+                          long long* rows) {
+  AttnParams p = {};
+  const fa_status st = check_common(p, B, H, H_kv, N, D, dtype, causal, -1.f, cu_seqlens,
+                                    max_seqlen, total_tokens);
+  if (st == FA_OK && rows != nullptr) *rows = p.total;
+  return st;
+}
+
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long rows,
                        unsigned long long cols, unsigned box_cols, unsigned box_rows) {
   EncodeTiledFn fn = encode_fn();

@@ -57,14 +57,18 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
                                     fa_dtype dtype, int causal, float scale,
                                     const int* cu_seqlens, int max_seqlen,
                                     long long total_tokens, fa_stream_t stream) {
-  if (B < 0 || N < 0 || H <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
-  const long long T = (cu_seqlens != nullptr) ? total_tokens : static_cast<long long>(B) * N;
-  if (T < 0) return FA_ERR_INVALID_ARG;
+  // The sizes are checked exactly as fa_bwd checks them (same status for the
+  // same mistake) before the scratch limit is applied.
+  long long T = 0;
+  const fa_status st = fa::check_bwd_sizes(B, H, H_kv, N, D, dtype, causal, cu_seqlens,
+                                           max_seqlen, total_tokens, &T);
+  if (st != FA_OK) return st;
   const size_t need = fa_bwd_workspace_size(T, H, D, dtype);
   if (need == 0) return FA_ERR_INVALID_ARG;
   if (need > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
-  if (fa::scratch_address(&scratch) != cudaSuccess) return FA_ERR_CUDA;
+  const cudaError_t e = fa::scratch_address(&scratch);
+  if (e != cudaSuccess) return fa::record_cuda(e);
   return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, D, dtype, causal, scale,
                 cu_seqlens, max_seqlen, total_tokens, scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
 }

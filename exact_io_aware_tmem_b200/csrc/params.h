@@ -136,6 +136,18 @@ cudaError_t launch_fp8_quantize(const void* x, void* x8, float* scale, int B, in
 // Decode partials (and the combine kernel when d.n_split > 1).
 cudaError_t launch_decode_bf16(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream);
 
+// Host: the argument checks fa_bwd applies to the sizes (status as fa_bwd
+// would return it); on success ``rows`` is the row count T of every tensor.
+// Declared with the C ABI's status type, which fa_api.cu and noalloc.cu see.
+#ifdef EXACT_IO_AWARE_TMEM_FA_H
+fa_status check_bwd_sizes(int B, int H, int H_kv, int N, int D, fa_dtype dtype, int causal,
+                          const int* cu_seqlens, int max_seqlen, long long total_tokens,
+                          long long* rows);
+// Host: FA_OK for cudaSuccess; otherwise FA_ERR_CUDA, with ``e`` kept as the
+// calling thread's last CUDA error (fa_last_cuda_error_string).
+fa_status record_cuda(cudaError_t e);
+#endif
+
 // Host: cuTensorMapEncodeTiled through the runtime's driver entry point.
 // Encodes a 2-D bf16 view [rows, cols] (row stride ``cols`` elements) with a
 // box of box_cols x box_rows and 128-byte swizzle. Returns false on failure.

@@ -53,6 +53,11 @@
  *   copies need it). Buffers are owned by the caller; the library allocates
  *   no device memory and keeps no per-call state (fa_bwd_noalloc's built-in
  *   scratch array is part of the loaded library, see its section).
+ * Device state: the library looks up, once per device and with that device
+ *   current, the device addresses of its own module variables (the error word
+ *   and fa_bwd_noalloc's scratch) and keeps them for the life of the process.
+ *   Do not use the library across a cudaDeviceReset, or from a context other
+ *   than the device's primary context: the kept addresses would be stale.
  * Streams: every entry point only enqueues work on ``stream`` (NULL = the
  *   legacy default stream) and returns without synchronising, except
  *   fa_check_device_error.
@@ -171,9 +176,12 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
  * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
  *
  * Arguments, layouts and results are those of fa_bwd without workspace and
- * ws_bytes. Limit: fa_bwd_workspace_size(T, H, D, dtype) must not exceed
- * FA_NOALLOC_SCRATCH_BYTES (about T * H * 4 bytes, so T * H <= 8,388,000);
- * larger problems return FA_ERR_UNSUPPORTED before anything is enqueued.
+ * ws_bytes. The sizes are checked as fa_bwd checks them first (same status
+ * for the same mistake). Limit: fa_bwd_workspace_size(T, H, D, dtype) must
+ * not exceed FA_NOALLOC_SCRATCH_BYTES (about T * H * 4 bytes, so
+ * T * H <= 8,388,000); larger problems return FA_ERR_UNSUPPORTED before
+ * anything is enqueued. A failed address lookup returns FA_ERR_CUDA and sets
+ * fa_last_cuda_error_string.
  *
  * The scratch is shared by every call on a device and keeps the last call's
  * contents; each call re-initialises what it reads. Calls whose kernels can

@@ -72,6 +72,23 @@ def test_peaks_fallback(monkeypatch, tmp_path):
     assert p["source"] == "fallback" and p["bf16_tflops"] == 1590.0 and p["hbm_gbs"] == 6650.0
 
 
+def test_tensor_peak_follows_length_of_timed_region():
+    peaks = {"bf16_tflops": 1644.9, "bf16_tflops_sustained": 1403.3}
+    # The driver's 20-step run lasts well under a second: burst clocks.
+    assert bench.tensor_peak(peaks, 0.15) == (1644.9, "burst")
+    # A seconds-long loop settles under the power cap.
+    assert bench.tensor_peak(peaks, 1.5) == (1403.3, "sustained")
+
+
+def test_default_workload_is_the_largest_single_gpu_configuration():
+    from exact_io_aware_tmem_b200.workloads import WORKLOADS, flops
+    w = WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert w.backward and w.D == 128 and w.N >= 4096
+    def work(x):
+        return sum(flops([x.N] * x.B, x.H, x.D, x.causal)) if not x.varlen else 0.0
+    assert work(w) == max(work(x) for x in WORKLOADS.values())
+
+
 def test_recorded_traffic_needs_matching_source(monkeypatch, tmp_path):
     (tmp_path / "profiles").mkdir()
     rec = {"bwd_dkdv_kernel": {"workload": "w", "source_sha": "stale", "bytes_per_launch": 5}}

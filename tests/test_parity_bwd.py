@@ -145,3 +145,24 @@ def test_bf16_workload_group_slice(name):
         ref_dv += rdv
     assert rel_fro(f64(dk[s0:s1, hk]), ref_dk) <= REL_BF16
     assert rel_fro(f64(dv[s0:s1, hk]), ref_dv) <= REL_BF16
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+def test_bf16_backward_deterministic(varlen):
+    """Two backward passes on the same inputs give the same bits: no step of
+    the bf16 backward accumulates through atomics or in a launch-dependent
+    order (dK / dV sum the GQA group in a fixed order inside one CTA, dQ is
+    written once per row)."""
+    lengths = [300, 129, 513] if varlen else [384, 384]
+    inp = random_case(21, dtype="bf16", lengths=lengths, H=4, H_kv=2, D=128, varlen=varlen)
+    B = len(lengths)
+    N = 0 if varlen else lengths[0]
+    a = to_api(inp, B, N)
+    kw = dict(causal=True, cu_seqlens=a.get("cu_seqlens"), max_seqlen=a.get("max_seqlen"))
+    o, lse = fa.fwd(a["q"], a["k"], a["v"], **kw)
+    first = fa.bwd(a["do"], a["q"], a["k"], a["v"], o, lse, **kw)
+    second = fa.bwd(a["do"], a["q"], a["k"], a["v"], o, lse, **kw)
+    st, where = fa.check_device_error()
+    assert st == 0, f"device error {st} at {where:#x}"
+    for name, x, y in zip(("dQ", "dK", "dV"), first, second):
+        assert torch.equal(x, y), name

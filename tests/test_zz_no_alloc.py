@@ -84,6 +84,7 @@ def _bwd_noalloc(lib, dev, o, lse, a):
 
 
 def _close(got, ref, dtype):
+    """Within the parity tolerance of the backward tests."""
     for g, r in zip(got, ref):
         g = g.double().cpu().numpy()
         r = r.double().cpu().numpy()
@@ -94,29 +95,44 @@ def _close(got, ref, dtype):
             assert np.abs(g - r).max() <= TOL_F32
 
 
+def _same_bits(got, ref):
+    """Both entry points run the same kernels, and the backward adds nothing
+    atomically, so the results must be identical; a difference would mean the
+    built-in scratch fed a kernel something the caller's workspace did not."""
+    for g, r in zip(got, ref):
+        assert torch.equal(g, r)
+
+
 CASES = [
     # (seed, dtype, lengths, H, H_kv, D, varlen, causal)
     (1, "bf16", [700, 700], 4, 2, 128, False, True),
     (2, "bf16", [5, 0, 300, 129], 4, 4, 64, True, False),
     (3, "f32", [130, 130], 2, 1, 64, False, True),
 ]
+# Run through fa_bwd_noalloc between a case's two calls, so the shared scratch
+# holds another problem's values when the second call starts.
+OTHER = (9, "bf16", [1000], 8, 8, 128, False, False)
 
 
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_twice_in_a_row(lib):
+    other = _problem(*OTHER)
+    _fwd(lib, *other)
     for case in CASES:
-        seed, dtype = case[0], case[1]
+        dtype = case[1]
         dev, o, lse, a = _problem(*case)
         _fwd(lib, dev, o, lse, a)
         ref = _bwd_with_workspace(lib, dev, o, lse, a)
         first = _bwd_noalloc(lib, dev, o, lse, a)
+        _bwd_noalloc(lib, *other)
         second = _bwd_noalloc(lib, dev, o, lse, a)
         torch.cuda.synchronize()
         where = ctypes.c_uint(0)
         assert lib.fa_check_device_error(None, ctypes.byref(where)) == _abi.FA_OK
         _close(first, ref, dtype)
         _close(second, ref, dtype)
-        assert seed
+        _same_bits(first, ref)
+        _same_bits(second, ref)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
@@ -128,3 +144,20 @@ def test_noalloc_rejects_problems_beyond_its_scratch(lib):
     st = lib.fa_bwd_noalloc(None, None, None, None, None, None, None, None, None, 1, H, H, T, D,
                             _abi.FA_BF16, 0, -1.0, None, 0, 0, None)
     assert st == _abi.FA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,D,dtype", [
+    (1, 6, 4, 9_000_000, 128, _abi.FA_BF16),    # H % H_kv != 0, and beyond the scratch
+    (1, 4, 4, 9_000_000, 96, _abi.FA_BF16),     # unsupported head dim, and beyond the scratch
+    (1, 4, 4, 1024, 128, 7),                    # unknown dtype
+    (-1, 4, 4, 1024, 128, _abi.FA_BF16),        # negative batch
+])
+def test_noalloc_reports_argument_errors_as_fa_bwd_does(lib, B, H, H_kv, N, D, dtype):
+    # Argument errors are found before any pointer is read or anything is
+    # enqueued, so null pointers are enough to compare the two statuses.
+    ref = lib.fa_bwd(None, None, None, None, None, None, None, None, None, B, H, H_kv, N, D,
+                     dtype, 0, -1.0, None, 0, 0, None, 0, None)
+    got = lib.fa_bwd_noalloc(None, None, None, None, None, None, None, None, None, B, H, H_kv,
+                             N, D, dtype, 0, -1.0, None, 0, 0, None)
+    assert ref != _abi.FA_OK
+    assert got == ref
