@@ -2,8 +2,9 @@
 """Attention forward + backward throughput on B200, one JSON line.
 
 A step is one pass of the whole hot path over one batch of the workload:
-fa_fwd (O, LSE) then fa_bwd (preprocess D_i, dK/dV kernel, dQ kernel), all
-through the C ABI of libfa_b200.so. Inputs are seeded
+fa_fwd (O, LSE) then fa_bwd (preprocess D_i and zero the dQ accumulator, the
+fused backward kernel, the dQ conversion), all through the C ABI of
+libfa_b200.so. Inputs are seeded
 synthetic Gaussians resident in HBM before the timed region starts.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
@@ -122,6 +123,7 @@ def source_sha(*names) -> str:
 
 
 KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "bwd_fused_kernel": ("bwd_fused.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "decode": ("fwd_bf16.cu", "common.cuh", "params.h"),
@@ -377,6 +379,7 @@ def run_ours(args, w) -> None:
                       dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.workspace_size(T, w.H, w.D, q.dtype), dtype=torch.uint8, device=dev)
+    ph = fa.BWD_FUSED  # preprocess (+ accumulator zeroing), fused kernel, dQ conversion
     bytes_in = sum(t.numel() * t.element_size() for t in (q, k, v, do))
 
     def step(ev=None):
@@ -385,13 +388,13 @@ def run_ours(args, w) -> None:
         fa.fwd(q, k, v, out=o, lse=lse, **kw)
         if ev is not None:
             ev[1].record()
-        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=1, **kw)
+        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph & 0x01, **kw)
         if ev is not None:
             ev[2].record()
-        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=2, **kw)
+        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph & 0x08, **kw)
         if ev is not None:
             ev[3].record()
-        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=4, **kw)
+        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph & 0x10, **kw)
         if ev is not None:
             ev[4].record()
 
@@ -430,7 +433,7 @@ def run_ours(args, w) -> None:
     max_ms = reduce_max(elapsed_ms, dev)
     k_ms = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
             for name, (a, b) in {"fwd_bf16_kernel": (0, 1), "bwd_preprocess": (1, 2),
-                                 "bwd_dkdv_kernel": (2, 3), "bwd_dq_kernel": (3, 4)}.items()}
+                                 "bwd_fused_kernel": (2, 3), "dq_convert": (3, 4)}.items()}
     k_ms = {n: reduce_max(t, dev) for n, t in k_ms.items()}
 
     # End to end through the public API with host buffers: pinned H2D of the
@@ -460,14 +463,13 @@ def run_ours(args, w) -> None:
     per_step_fl = fwd_fl + bwd_fl
     value = aggregate(per_step_fl * args.steps, world, [max_ms / 1e3]) / 1e12
     fwd_tf = fwd_fl / (k_ms["fwd_bf16_kernel"] / 1e3) / 1e12
-    bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_dkdv_kernel"] + k_ms["bwd_dq_kernel"]
+    bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_fused_kernel"] + k_ms["dq_convert"]
     bwd_tf = bwd_fl / (bwd_ms / 1e3) / 1e12
     # Dominant kernel: the one with the largest share of the step. Algorithmic
-    # FLOPs per launch: the forward's two products (4 N^2 D per head), the
-    # dK/dV kernel's four (S, dP, dV, dK: 8 N^2 D), the dQ kernel's three
-    # (S, dP again and dQ: 6 N^2 D), causal halving each.
-    kernel_fl = {"fwd_bf16_kernel": fwd_fl, "bwd_dkdv_kernel": 2.0 * fwd_fl,
-                 "bwd_dq_kernel": 1.5 * fwd_fl}
+    # FLOPs per launch: the forward's two products (4 N^2 D per head) and the
+    # fused backward's five (S, dP, dV, dK, dQ: 10 N^2 D, the method's 2.5x),
+    # causal halving each.
+    kernel_fl = {"fwd_bf16_kernel": fwd_fl, "bwd_fused_kernel": bwd_fl}
     dom = max(kernel_fl, key=lambda n: k_ms[n])
     dom_fl = kernel_fl[dom]
     achieved = dom_fl / (k_ms[dom] / 1e3) / 1e12

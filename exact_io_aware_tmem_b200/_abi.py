@@ -18,6 +18,14 @@ FA_ERR_CUDA = 3
 FA_ERR_DEVICE_TIMEOUT = 4
 FA_BF16 = 0
 FA_F32 = 1
+# Backward phase bits (include/fa.h FA_BWD_PHASE_*) and the two whole passes.
+BWD_PREPROCESS = 0x01
+BWD_DKDV = 0x02
+BWD_DQ = 0x04
+BWD_FUSED_KERNEL = 0x08
+BWD_DQ_CONVERT = 0x10
+BWD_SPLIT = 0x07
+BWD_FUSED = 0x19
 
 c_void_p = ctypes.c_void_p
 c_int = ctypes.c_int
@@ -30,6 +38,7 @@ SIGNATURES = {
     "fa_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                        c_int, c_int, c_int, c_int, c_float, c_void_p, c_int, c_ll, c_void_p]),
     "fa_bwd_workspace_size": (c_size_t, [c_ll, c_int, c_int, c_int]),
+    "fa_bwd_phases_workspace_size": (c_size_t, [ctypes.c_uint, c_ll, c_int, c_int, c_int]),
     "fa_bwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                        c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                        c_float, c_void_p, c_int, c_ll, c_void_p, c_size_t, c_void_p]),

@@ -73,8 +73,13 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = Fal
     return out, lse
 
 
-def workspace_size(T: int, H: int, D: int, dtype: torch.dtype) -> int:
-    return int(_abi.lib().fa_bwd_workspace_size(T, H, D, _DTYPES[dtype]))
+BWD_FUSED = _abi.BWD_FUSED
+BWD_SPLIT = _abi.BWD_SPLIT
+
+
+def workspace_size(T: int, H: int, D: int, dtype: torch.dtype, phases: int = BWD_FUSED) -> int:
+    """Bytes of backward workspace for ``phases`` (fa_bwd_phases_workspace_size)."""
+    return int(_abi.lib().fa_bwd_phases_workspace_size(int(phases), T, H, D, _DTYPES[dtype]))
 
 
 def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -82,11 +87,14 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
         max_seqlen: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
         dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
-        dv: Optional[torch.Tensor] = None, phases: int = 7):
+        dv: Optional[torch.Tensor] = None, phases: int = BWD_FUSED):
     """Attention backward for the loss sum(O * dO). Returns (dQ, dK, dV).
 
-    ``phases`` selects the kernels to enqueue (bit 0 the D_i preprocess, bit 1
-    the dK / dV kernel, bit 2 the dQ kernel); the default runs all three.
+    ``phases`` selects the kernels to enqueue (the FA_BWD_PHASE_* bits of
+    include/fa.h): the default ``BWD_FUSED`` runs the preprocess, the fused
+    kernel and the dQ conversion; ``BWD_SPLIT`` runs the preprocess, the
+    dK / dV kernel and the dQ kernel (bitwise reproducible dQ, smaller
+    workspace); single bits enqueue one kernel, to time it.
     """
     B, N, H, H_kv, D, max_sl, T = _shape(q, k, cu_seqlens, max_seqlen)
     for t in (dout, o, v, lse):
@@ -95,7 +103,7 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    need = workspace_size(T, H, D, q.dtype)
+    need = workspace_size(T, H, D, q.dtype, phases)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     s = -1.0 if scale is None else float(scale)

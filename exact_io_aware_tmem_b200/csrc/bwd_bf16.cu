@@ -95,7 +95,8 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
 
 // ------------------------------------------------------------ preprocess ---
 
-// One warp per (token, head) row: D_i = dO_i . O_i into delta [H, T].
+// One warp per (token, head) row: D_i = dO_i . O_i into delta [H, T], and,
+// for the fused backward, the row's dQ accumulator set to zero.
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnParams p) {
   const long long rows = p.total * p.H;
   const int lane = threadIdx.x % 32;
@@ -116,6 +117,9 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const AttnParams p)
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(FULL, acc, s);
     if (lane == 0) p.delta[static_cast<size_t>(h) * p.total + tok] = acc;
+    if (p.dq_accum != nullptr)
+      for (int d = 4 * lane; d < p.D; d += 128)
+        *reinterpret_cast<float4*>(p.dq_accum + off + d) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 

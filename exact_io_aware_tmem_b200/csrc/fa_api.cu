@@ -353,11 +353,20 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v, const float*
   return fa::cuda_status(fa::launch_fwd_fp8(p, f, s));
 }
 
-size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype) {
+size_t fa_bwd_phases_workspace_size(unsigned mask, long long total_tokens, int H, int D,
+                                    fa_dtype dtype) {
   if (total_tokens < 0 || H <= 0 || D <= 0) return 0;
   if (dtype != FA_BF16 && dtype != FA_F32) return 0;
+  if (mask == 0 || (mask & ~FA_BWD_ALL) != 0) return 0;
   const size_t T = static_cast<size_t>(total_tokens);
-  return fa::round256(T * H * sizeof(float)) + 256;
+  const size_t delta = fa::round256(T * H * sizeof(float));
+  // The fused kernel and the dQ conversion also need the fp32 dQ accumulator.
+  const bool acc = dtype == FA_BF16 && (mask & (FA_BWD_PHASE_FUSED | FA_BWD_PHASE_DQ_CONVERT));
+  return delta + (acc ? fa::round256(T * H * D * sizeof(float)) : 0) + 256;
+}
+
+size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype) {
+  return fa_bwd_phases_workspace_size(FA_BWD_FUSED, total_tokens, H, D, dtype);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -365,8 +374,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int D, fa_dtype dtype, int causal, float scale, const int* cu_seqlens,
                  int max_seqlen, long long total_tokens, void* workspace, size_t ws_bytes,
                  fa_stream_t stream) {
-  return fa_bwd_phases(7u, q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, D, dtype, causal,
-                       scale, cu_seqlens, max_seqlen, total_tokens, workspace, ws_bytes, stream);
+  return fa_bwd_phases(FA_BWD_FUSED, q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, D, dtype,
+                       causal, scale, cu_seqlens, max_seqlen, total_tokens, workspace, ws_bytes,
+                       stream);
 }
 
 fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void* v,
@@ -374,8 +384,9 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
                         void* dv, int B, int H, int H_kv, int N, int D, fa_dtype dtype, int causal,
                         float scale, const int* cu_seqlens, int max_seqlen, long long total_tokens,
                         void* workspace, size_t ws_bytes, fa_stream_t stream) {
-  if (mask == 0 || mask > 7u) return FA_ERR_INVALID_ARG;
-  if (dtype == FA_F32 && mask != 7u) return FA_ERR_UNSUPPORTED;
+  if (mask == 0 || (mask & ~FA_BWD_ALL) != 0) return FA_ERR_INVALID_ARG;
+  // The fp32 path is one backward of its own: only the two whole-pass masks.
+  if (dtype == FA_F32 && mask != FA_BWD_FUSED && mask != FA_BWD_SPLIT) return FA_ERR_UNSUPPORTED;
   AttnParams p = {};
   fa_status st = fa::check_common(p, B, H, H_kv, N, D, dtype, causal, scale, cu_seqlens,
                                   max_seqlen, total_tokens);
@@ -387,7 +398,8 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
   for (const void* ptr : ptrs)
     if (!fa::aligned16(ptr)) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
-  if (ws_bytes < fa_bwd_workspace_size(p.total, H, D, dtype)) return FA_ERR_INVALID_ARG;
+  if (ws_bytes < fa_bwd_phases_workspace_size(mask, p.total, H, D, dtype))
+    return FA_ERR_INVALID_ARG;
   p.q = q;
   p.k = k;
   p.v = v;
@@ -398,11 +410,25 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
   p.dk = dk;
   p.dv = dv;
   p.delta = static_cast<float*>(workspace);
+  // The accumulator follows the D_i rows whenever the workspace holds it, so
+  // that a preprocess enqueued on its own (bit 0 alone) zeroes it for a fused
+  // kernel enqueued by a later call on the same workspace.
+  const size_t delta_bytes = fa::round256(static_cast<size_t>(p.total) * H * sizeof(float));
+  const size_t acc_bytes = static_cast<size_t>(p.total) * H * D * sizeof(float);
+  if (dtype == FA_BF16 && ws_bytes >= delta_bytes + acc_bytes)
+    p.dq_accum = reinterpret_cast<float*>(static_cast<char*>(workspace) + delta_bytes);
   p.err.word = fa::err_word();
   if (p.err.word == nullptr) return FA_ERR_CUDA;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e =
-      (dtype == FA_F32) ? fa::launch_bwd_f32(p, s) : fa::launch_bwd_bf16(p, s, mask);
+  cudaError_t e = cudaSuccess;
+  if (dtype == FA_F32) {
+    e = fa::launch_bwd_f32(p, s);
+  } else {
+    if (mask & (FA_BWD_PHASE_PREPROCESS | FA_BWD_PHASE_DKDV | FA_BWD_PHASE_DQ))
+      e = fa::launch_bwd_bf16(p, s, mask & 7u);
+    if (e == cudaSuccess && (mask & FA_BWD_PHASE_FUSED)) e = fa::launch_bwd_fused(p, s);
+    if (e == cudaSuccess && (mask & FA_BWD_PHASE_DQ_CONVERT)) e = fa::launch_dq_convert(p, s);
+  }
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return fa::cuda_status(e);
 }

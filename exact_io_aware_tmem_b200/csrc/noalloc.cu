@@ -63,12 +63,16 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
   const fa_status st = fa::check_bwd_sizes(B, H, H_kv, N, D, dtype, causal, cu_seqlens,
                                            max_seqlen, total_tokens, &T);
   if (st != FA_OK) return st;
-  const size_t need = fa_bwd_workspace_size(T, H, D, dtype);
+  // The split backward needs only the D_i rows as scratch (the fused one
+  // would also need a T x H x D fp32 dQ accumulator).
+  const size_t need = fa_bwd_phases_workspace_size(FA_BWD_SPLIT, T, H, D, dtype);
   if (need == 0) return FA_ERR_INVALID_ARG;
   if (need > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   const cudaError_t e = fa::scratch_address(&scratch);
   if (e != cudaSuccess) return fa::record_cuda(e);
-  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, D, dtype, causal, scale,
-                cu_seqlens, max_seqlen, total_tokens, scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
+  // ws_bytes = need (not the array's size), so the path never takes the
+  // scratch for a dQ accumulator.
+  return fa_bwd_phases(FA_BWD_SPLIT, q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, D, dtype,
+                       causal, scale, cu_seqlens, max_seqlen, total_tokens, scratch, need, stream);
 }

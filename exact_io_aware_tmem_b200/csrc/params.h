@@ -21,6 +21,7 @@ struct AttnParams {
   void* dk;
   void* dv;
   float* delta;     // fp32 [H, T]: D_i = dO_i . O_i (backward workspace)
+  float* dq_accum;  // fp32 [T, H, D] dQ accumulator of the fused backward, or null
   const int* cu_seqlens;  // null for dense batches
   int B, H, H_kv, N, D;
   int causal;
@@ -125,8 +126,13 @@ struct Fp8Args {
 cudaError_t launch_fwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream);
-// mask: bit 0 preprocess (D_i), bit 1 dK/dV kernel, bit 2 dQ kernel.
+// mask: bit 0 preprocess (D_i, and zeroes dq_accum when it is set), bit 1
+// dK/dV kernel, bit 2 dQ kernel (the split backward).
 cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned mask);
+// The fused backward (every product once; dQ added into p.dq_accum) and the
+// conversion dQ = bf16(scale * dq_accum).
+cudaError_t launch_bwd_fused(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_dq_convert(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
 // E4M3 forward (D = 128) on codes from launch_fp8_quantize.
 cudaError_t launch_fwd_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream);

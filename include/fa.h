@@ -115,11 +115,37 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  fa_stream_t stream);
 
 /*
- * fa_bwd_workspace_size - bytes of device scratch fa_bwd needs for T tokens
- * and H query heads: the float32 row terms D_i = dO_i . O_i [H, T], rounded
- * up to 256 bytes, plus 256. D is checked but does not change the size.
- * Returns 0 for invalid sizes.
+ * Backward phases. fa_bwd enqueues FA_BWD_FUSED: the preprocess, the fused
+ * kernel that forms every product of the method once per (query tile, key
+ * tile) pair and adds the dQ partials into an fp32 accumulator, and the dQ
+ * conversion. FA_BWD_SPLIT is the same backward as two kernels that share
+ * no accumulator: one for dK / dV and one for dQ, which recomputes S and dP
+ * (seven products per tile pair instead of five). It needs less workspace and
+ * gives bitwise reproducible dQ; the fused path's dQ is reproducible only to
+ * rounding, because the order of its fp32 additions over key tiles is not
+ * fixed (dK and dV are reproducible on both paths).
  */
+#define FA_BWD_PHASE_PREPROCESS 0x01u /* D_i = dO_i . O_i; zeroes the dQ accumulator */
+#define FA_BWD_PHASE_DKDV 0x02u       /* split path: dK, dV                          */
+#define FA_BWD_PHASE_DQ 0x04u         /* split path: dQ                              */
+#define FA_BWD_PHASE_FUSED 0x08u      /* fused path: dK, dV, dQ accumulator          */
+#define FA_BWD_PHASE_DQ_CONVERT 0x10u /* fused path: dQ = bf16(scale * accumulator)  */
+#define FA_BWD_SPLIT 0x07u
+#define FA_BWD_FUSED 0x19u
+#define FA_BWD_ALL 0x1Fu
+
+/*
+ * fa_bwd_phases_workspace_size - bytes of device scratch fa_bwd_phases needs
+ * for ``mask``, T tokens and H query heads: the float32 row terms
+ * D_i = dO_i . O_i [H, T], rounded up to 256 bytes, plus, for bf16 when the
+ * mask has FA_BWD_PHASE_FUSED or FA_BWD_PHASE_DQ_CONVERT, the float32 dQ
+ * accumulator [T, H, D] rounded up to 256 bytes; plus 256. Returns 0 for
+ * invalid sizes or masks.
+ *
+ * fa_bwd_workspace_size - the same for fa_bwd (mask FA_BWD_FUSED).
+ */
+size_t fa_bwd_phases_workspace_size(unsigned mask, long long total_tokens, int H, int D,
+                                    fa_dtype dtype);
 size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtype);
 
 /*
@@ -132,7 +158,7 @@ size_t fa_bwd_workspace_size(long long total_tokens, int H, int D, fa_dtype dtyp
  *   dQ = scale dS K, dK = scale dS^T Q
  * (the relations the "Flash Attention self-test", section D, asks for). With
  * grouped-query attention dk and dv of a key/value head are summed over the
- * query heads that share it.
+ * query heads that share it. Runs the FA_BWD_FUSED phases.
  *
  *   q, k, v, o, lse, dout   inputs, as written / read by fa_fwd
  *   dq, dk, dv              outputs, same dtype and layout as q, k, v
@@ -150,12 +176,16 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  fa_stream_t stream);
 
 /*
- * fa_bwd_phases - fa_bwd restricted to some of its three kernels, so that
- * each can be timed by itself: bit 0 = preprocess (D_i = dO_i . O_i into the
- * workspace), bit 1 = the dK / dV kernel, bit 2 = the dQ kernel (bits 1 and 2
- * both read D_i, so bit 0 must have run on the same workspace first).
- * fa_bwd(...) is fa_bwd_phases(7, ...). For FA_F32 only mask 7 is accepted
- * (FA_ERR_UNSUPPORTED otherwise). Other arguments as for fa_bwd.
+ * fa_bwd_phases - fa_bwd restricted to the phases in ``mask`` (the
+ * FA_BWD_PHASE_* bits), enqueued in bit order; FA_BWD_SPLIT selects the
+ * split backward, and single bits let each kernel be timed by itself. Every
+ * phase after the preprocess reads D_i, so the preprocess must have run on
+ * the same workspace first; it also zeroes the dQ accumulator whenever the
+ * workspace is large enough to hold one (bf16), which the fused kernel
+ * requires. ws_bytes must be at least
+ * fa_bwd_phases_workspace_size(mask, T, H, D, dtype). For FA_F32 only the
+ * masks FA_BWD_FUSED and FA_BWD_SPLIT are accepted (both run the one fp32
+ * backward; FA_ERR_UNSUPPORTED otherwise). Other arguments as for fa_bwd.
  */
 fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void* v,
                         const void* o, const float* lse, const void* dout, void* dq, void* dk,
@@ -175,12 +205,15 @@ fa_status fa_bwd_phases(unsigned mask, const void* q, const void* k, const void*
  * device memory that every GPU loading the library holds until the process
  * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
  *
- * Arguments, layouts and results are those of fa_bwd without workspace and
- * ws_bytes. The sizes are checked as fa_bwd checks them first (same status
- * for the same mistake). Limit: fa_bwd_workspace_size(T, H, D, dtype) must
- * not exceed FA_NOALLOC_SCRATCH_BYTES (about T * H * 4 bytes, so
- * T * H <= 8,388,000); larger problems return FA_ERR_UNSUPPORTED before
- * anything is enqueued. A failed address lookup returns FA_ERR_CUDA and sets
+ * Arguments and layouts are those of fa_bwd without workspace and ws_bytes.
+ * It runs the split backward (FA_BWD_SPLIT), whose only scratch is the D_i
+ * rows, so its results are identical to fa_bwd_phases(FA_BWD_SPLIT, ...)
+ * and agree with fa_bwd within rounding. The sizes are checked as fa_bwd
+ * checks them first (same status for the same mistake). Limit:
+ * fa_bwd_phases_workspace_size(FA_BWD_SPLIT, T, H, D, dtype) must not exceed
+ * FA_NOALLOC_SCRATCH_BYTES (about T * H * 4 bytes, so T * H <= 8,388,000);
+ * larger problems return FA_ERR_UNSUPPORTED before anything is enqueued. A
+ * failed address lookup returns FA_ERR_CUDA and sets
  * fa_last_cuda_error_string.
  *
  * The scratch is shared by every call on a device and keeps the last call's

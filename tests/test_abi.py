@@ -45,9 +45,16 @@ def test_version_and_error_strings(lib):
 def test_workspace_size(lib):
     T, H, D = 1000, 16, 128
     r = lambda x: (x + 255) // 256 * 256
-    assert lib.fa_bwd_workspace_size(T, H, D, _abi.FA_BF16) == r(T * H * 4) + 256
+    # fa_bwd (fused): D_i rows plus the fp32 dQ accumulator for bf16.
+    assert lib.fa_bwd_workspace_size(T, H, D, _abi.FA_BF16) == r(T * H * 4) + r(T * H * D * 4) + 256
     assert lib.fa_bwd_workspace_size(T, H, D, _abi.FA_F32) == r(T * H * 4) + 256
     assert lib.fa_bwd_workspace_size(-1, H, D, _abi.FA_BF16) == 0
+    ws = lib.fa_bwd_phases_workspace_size
+    assert ws(_abi.BWD_SPLIT, T, H, D, _abi.FA_BF16) == r(T * H * 4) + 256
+    assert ws(_abi.BWD_FUSED, T, H, D, _abi.FA_BF16) == lib.fa_bwd_workspace_size(T, H, D, 0)
+    assert ws(_abi.BWD_DQ_CONVERT, T, H, D, _abi.FA_BF16) == r(T * H * 4) + r(T * H * D * 4) + 256
+    assert ws(0, T, H, D, _abi.FA_BF16) == 0
+    assert ws(0x20, T, H, D, _abi.FA_BF16) == 0
 
 
 def _fwd(lib, **kw):
@@ -94,6 +101,24 @@ def test_bwd_rejects_small_workspace(lib):
     args[-3] = 100  # workspace must be 256-byte aligned
     args[-2] = need
     assert lib.fa_bwd(*args) == _abi.FA_ERR_INVALID_ARG
+
+
+def test_bwd_phases_rejects_bad_masks(lib):
+    need = lib.fa_bwd_workspace_size(8, 2, 64, _abi.FA_BF16)
+
+    def call(mask, dtype=_abi.FA_BF16):
+        return lib.fa_bwd_phases(mask, *([256] * 9), 1, 2, 2, 8, 64, dtype, 0, 0.0, None, 0, 0,
+                                 256, need, None)
+    assert call(0) == _abi.FA_ERR_INVALID_ARG
+    assert call(0x20) == _abi.FA_ERR_INVALID_ARG
+    # The fp32 backward is one pass: its phases cannot be enqueued one by one.
+    assert call(_abi.BWD_FUSED_KERNEL, _abi.FA_F32) == _abi.FA_ERR_UNSUPPORTED
+    assert call(_abi.BWD_DKDV, _abi.FA_F32) == _abi.FA_ERR_UNSUPPORTED
+    # The split path needs only the D_i rows; a fused mask needs the accumulator.
+    small = lib.fa_bwd_phases_workspace_size(_abi.BWD_SPLIT, 8, 2, 64, _abi.FA_BF16)
+    assert small < need
+    args = [*([256] * 9), 1, 2, 2, 8, 64, _abi.FA_BF16, 0, 0.0, None, 0, 0, 256, small, None]
+    assert lib.fa_bwd_phases(_abi.BWD_FUSED, *args) == _abi.FA_ERR_INVALID_ARG
 
 
 def test_no_gpu_reports_cuda_error_not_crash(lib):

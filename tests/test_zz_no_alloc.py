@@ -60,14 +60,16 @@ def _grads(dev):
             torch.full_like(dev["v"], float("nan")))
 
 
-def _bwd_with_workspace(lib, dev, o, lse, a):
+def _bwd_with_workspace(lib, dev, o, lse, a, mask):
+    """fa_bwd_phases(mask) with a caller-allocated workspace."""
     dq, dk, dv = _grads(dev)
-    need = lib.fa_bwd_workspace_size(a["T"], a["H"], a["D"], a["dtype"])
+    need = lib.fa_bwd_phases_workspace_size(mask, a["T"], a["H"], a["D"], a["dtype"])
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
-    st = lib.fa_bwd(_p(dev["q"]), _p(dev["k"]), _p(dev["v"]), _p(o), _p(lse), _p(dev["do"]),
-                    _p(dq), _p(dk), _p(dv), a["B"], a["H"], a["H_kv"], a["N"], a["D"], a["dtype"],
-                    a["causal"], -1.0, None if a["cu"] is None else _p(a["cu"]), a["max_seqlen"],
-                    a["T"], _p(ws), need, None)
+    st = lib.fa_bwd_phases(mask, _p(dev["q"]), _p(dev["k"]), _p(dev["v"]), _p(o), _p(lse),
+                           _p(dev["do"]), _p(dq), _p(dk), _p(dv), a["B"], a["H"], a["H_kv"],
+                           a["N"], a["D"], a["dtype"], a["causal"], -1.0,
+                           None if a["cu"] is None else _p(a["cu"]), a["max_seqlen"], a["T"],
+                           _p(ws), need, None)
     assert st == _abi.FA_OK
     return dq, dk, dv
 
@@ -96,9 +98,10 @@ def _close(got, ref, dtype):
 
 
 def _same_bits(got, ref):
-    """Both entry points run the same kernels, and the backward adds nothing
-    atomically, so the results must be identical; a difference would mean the
-    built-in scratch fed a kernel something the caller's workspace did not."""
+    """fa_bwd_noalloc runs the split backward's kernels, which add nothing
+    atomically, so its results must be identical to the split backward run
+    with a caller workspace; a difference would mean the built-in scratch fed
+    a kernel something the caller's workspace did not."""
     for g, r in zip(got, ref):
         assert torch.equal(g, r)
 
@@ -122,7 +125,8 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row(lib):
         dtype = case[1]
         dev, o, lse, a = _problem(*case)
         _fwd(lib, dev, o, lse, a)
-        ref = _bwd_with_workspace(lib, dev, o, lse, a)
+        ref = _bwd_with_workspace(lib, dev, o, lse, a, _abi.BWD_FUSED)       # fa_bwd's path
+        ref_split = _bwd_with_workspace(lib, dev, o, lse, a, _abi.BWD_SPLIT)
         first = _bwd_noalloc(lib, dev, o, lse, a)
         _bwd_noalloc(lib, *other)
         second = _bwd_noalloc(lib, dev, o, lse, a)
@@ -131,15 +135,15 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row(lib):
         assert lib.fa_check_device_error(None, ctypes.byref(where)) == _abi.FA_OK
         _close(first, ref, dtype)
         _close(second, ref, dtype)
-        _same_bits(first, ref)
-        _same_bits(second, ref)
+        _same_bits(first, ref_split)
+        _same_bits(second, ref_split)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
     # T * H * 4 bytes > 32 MiB: refused before anything is enqueued (no pointer
     # is touched, so none is needed).
     T, H, D = 9_000_000, 1, 128
-    need = lib.fa_bwd_workspace_size(T, H, D, _abi.FA_BF16)
+    need = lib.fa_bwd_phases_workspace_size(_abi.BWD_SPLIT, T, H, D, _abi.FA_BF16)
     assert need > SCRATCH_BYTES
     st = lib.fa_bwd_noalloc(None, None, None, None, None, None, None, None, None, 1, H, H, T, D,
                             _abi.FA_BF16, 0, -1.0, None, 0, 0, None)
