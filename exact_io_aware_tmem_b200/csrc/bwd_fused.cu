@@ -18,14 +18,20 @@
 //     dP^T = V dO_t^T           (A, B in shared memory)         -> TMEM dP
 //     dV  += P^T dO_t           (A = P^T, bf16 in TMEM over S)  -> TMEM dV
 //     dK  += dS^T Q_t           (A = dS^T, bf16 in TMEM over dP) -> TMEM dK
-//     dQ_t = dS K               (A = dS, read MN-major from the swizzled
-//                                dS^T tile the dS warps also write to shared
-//                                memory; queries on the TMEM lanes)
+//     dQ_t^T = K^T dS^T         (D = 128; A = K^T and B = dS^T read MN-major
+//                                from the K tile and from a swizzled dS^T
+//                                tile the dS warps also write to shared
+//                                memory; head dim on the TMEM lanes)
+//     dQ_t = dS K               (D = 64; the same tiles, queries on the lanes)
 // and the fp32 dQ_t partial is added into the caller's fp32 accumulator
 // dQacc [T, H, D] (zeroed by the preprocess kernel; a convert kernel writes
-// dQ = bf16(scale dQacc) afterwards). The accumulation order over key tiles
-// is not fixed, so dQ is reproducible only to rounding; dK and dV are summed
-// in a fixed order inside one CTA.
+// dQ = bf16(scale dQacc) afterwards). With the head dim on the lanes, one
+// warp-wide reduction for one query covers 32 consecutive entries of its
+// accumulator row (a whole 128-byte line): at 64 KB of partials per step, the
+// line-per-instruction form is what keeps the additions at the L2's rate
+// (about twice that of one 16-byte piece of a different row per lane). The
+// accumulation order over key tiles is not fixed, so dQ is reproducible only
+// to rounding; dK and dV are summed in a fixed order inside one CTA.
 //
 // TMEM columns: S [0,128), dP [128,256), dV, dK after them. At D = 128 the
 // 512 columns are full, so dQ_t is formed over dP once dK_t has read dS^T
@@ -36,7 +42,8 @@
 //   warps 0-7  dS warps. Thread = key row (TMEM lane) for S^T / dP^T, warps w
 //              and w+4 taking query columns [64 hf, 64 hf + 64). Per step:
 //              exponentials of S^T_t -> P^T_t into TMEM; then the read-out of
-//              dQ_{t-1} (thread = query row) and its addition into dQacc;
+//              dQ_{t-1} (thread = head-dim entry at D = 128, query row at
+//              D = 64) and its addition into dQacc;
 //              then dS^T_t into TMEM and into the shared dS tile.
 //   warp 8     TMA producer: K, V once; Q_t (with the step's LSE and D_i
 //              staged beside it) and dO_t through two-stage rings.
@@ -73,6 +80,10 @@ struct Cfg {
   static constexpr int QS = 2;                       // Q stages (with LSE, D_i)
   static constexpr int GS = 2;                       // dO stages
   static constexpr bool ALIAS = D == 128;            // dQ_t formed over dP
+  // D = 128: the product is dQ_t^T = K^T dS^T, head dim on the TMEM lanes, so
+  // that one warp-wide add covers 32 consecutive head-dim entries of a query
+  // row: a whole 128-byte line of the accumulator per instruction.
+  static constexpr bool DQT = D == 128;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr uint32_t TM_DQ = ALIAS ? TM_DP : 256 + 2 * D;
   static constexpr uint32_t OFF_K = 0;
@@ -124,7 +135,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
   return __all_sync(FULL, ok);
 }
 
-// One 128-row tile of a token-major tensor (its CH 64-column blocks).
+// One 128-row tile of a token-major tensor (its D / 64 column blocks).
 template <int D>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                           int head, int row) {
@@ -150,8 +161,13 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
   }
 }
 
-// dst[0..31] += a[0..31] (fp32, global, relaxed reduction at GPU scope; the
-// accumulator is only read by a later kernel).
+// *dst += x (fp32, global, relaxed reduction at GPU scope; the accumulator is
+// only read by a later kernel).
+__device__ __forceinline__ void red_add(float* dst, float x) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(dst), "f"(x) : "memory");
+}
+
+// dst[0..31] += a[0..31], as above.
 __device__ __forceinline__ void red_add_row32(float* dst, const uint32_t (&a)[32]) {
 #pragma unroll
   for (int v = 0; v < 8; ++v)
@@ -295,7 +311,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t leader = elect_one();
     constexpr uint32_t ID_SDP = idesc_bf16(BT, BT, false, false);  // S^T, dP^T
     constexpr uint32_t ID_KV = idesc_bf16(BT, D, false, true);     // dV, dK (A from TMEM)
-    constexpr uint32_t ID_DQ = idesc_bf16(BT, D, true, true);      // dQ_t = dS K
+    constexpr uint32_t ID_DQ = C::DQT ? idesc_bf16(D, BT, true, true)    // dQ_t^T = K^T dS^T
+                                      : idesc_bf16(BT, D, true, true);   // dQ_t = dS K
     const uint64_t k_kmaj = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
     const uint64_t v_kmaj = sdesc_sw128(sbase + C::OFF_V, 16, 1024);
     const uint64_t q_kmaj = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
@@ -371,9 +388,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
       }
 #pragma unroll
-      for (int kk = 0; kk < BT / 16; ++kk)
-        mma_ss_if(leader, tmem + C::TM_DQ, sdesc_add(ds_mn, kk * 2048), sdesc_add(k_mn, kk * 2048),
-                  ID_DQ, kk > 0);
+      for (int kk = 0; kk < BT / 16; ++kk) {
+        // K-dim = 128 keys in steps of 16 (16 rows of both tiles).
+        const uint64_t ds = sdesc_add(ds_mn, kk * 2048), kt = sdesc_add(k_mn, kk * 2048);
+        if constexpr (C::DQT)
+          mma_ss_if(leader, tmem + C::TM_DQ, kt, ds, ID_DQ, kk > 0);
+        else
+          mma_ss_if(leader, tmem + C::TM_DQ, ds, kt, ID_DQ, kk > 0);
+      }
       tc_commit_if(leader, bars.dq_full());
       if (more) {
         if (C::ALIAS) {
@@ -410,26 +432,53 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* ds_row = smem + C::OFF_DS + hf * SPAN + r * 128;
     float* const dq_acc = p.dq_accum;
 
-    // Adds dQ_tq (the dQ partial of step tq, in TMEM) into dQacc.
+    // Adds the dQ partial of step tq (in TMEM) into dQacc.
     auto drain_dq = [&](int tq) -> bool {
       if (!warp_wait(bars.dq_full(), tq & 1, p.err, abort, W_DQFULL)) return false;
       tc_fence_after();
-      constexpr int NC = D / 64;   // 32-column blocks per thread
+      constexpr int NC = C::DQT ? 2 : D / 64;   // 32-column blocks per thread
       uint32_t a[NC][32];
 #pragma unroll
       for (int c = 0; c < NC; ++c)
-        tmem_ld32(tmem + lane_off + C::TM_DQ + hf * (D / 2) + 32 * c, a[c]);
+        tmem_ld32(tmem + lane_off + C::TM_DQ + hf * (32 * NC) + 32 * c, a[c]);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < NC; ++c) reg_fence(a[c]);
       tc_fence_before();
       mbar_arrive(bars.dq_free());
       const int h = hk * g + tq / n_qt;
-      const int qpos = (i0 + tq % n_qt) * BT + (warp & 3) * 32 + lane;
-      if (qpos < sq.len) {
-        float* dst = dq_acc + (static_cast<size_t>(sq.start + qpos) * p.H + h) * D + hf * (D / 2);
+      const int qtile = (i0 + tq % n_qt) * BT;
+      if constexpr (C::DQT) {
+        // Thread = head-dim entry d (TMEM lane); columns = queries
+        // [64 hf, 64 hf + 64) of the tile. Query q's row of dQacc starts at
+        // ((start + q) H + h) D; the warp's 32 lanes are 32 consecutive d.
+        const int d = (warp & 3) * 32 + lane;
+        const int q0 = qtile + 64 * hf;
+        const size_t row_step = static_cast<size_t>(p.H) * D;
+        float* col = dq_acc + static_cast<size_t>(sq.start + q0) * row_step +
+                     static_cast<size_t>(h) * D + d;
+        const int nq = min(64, sq.len - q0);   // valid queries of this half (warp-uniform)
+        if (nq >= 64) {
 #pragma unroll
-        for (int c = 0; c < NC; ++c) red_add_row32(dst + 32 * c, a[c]);
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              red_add(col + (32 * c + i) * row_step, __uint_as_float(a[c][i]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (32 * c + i < nq) red_add(col + (32 * c + i) * row_step, __uint_as_float(a[c][i]));
+        }
+      } else {
+        // Thread = query row (TMEM lane), columns [hf D / 2, hf D / 2 + D / 2).
+        const int qpos = qtile + (warp & 3) * 32 + lane;
+        if (qpos < sq.len) {
+          float* dst = dq_acc + (static_cast<size_t>(sq.start + qpos) * p.H + h) * D + hf * (D / 2);
+#pragma unroll
+          for (int c = 0; c < NC; ++c) red_add_row32(dst + 32 * c, a[c]);
+        }
       }
       return true;
     };

@@ -893,7 +893,7 @@ cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream
 
 cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream) {
   if (p.D == 64) return launch_d<64>(p, stream);
-  if (p.D == 128) return launch_d<128>(p, stream);
+  if (p.D == 128) return launch_fwd_pair(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -126,6 +126,8 @@ struct Fp8Args {
 cudaError_t launch_fwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream);
+// The D = 128 forward with two query tiles per CTA (launch_fwd_bf16 uses it).
+cudaError_t launch_fwd_pair(const AttnParams& p, cudaStream_t stream);
 // mask: bit 0 preprocess (D_i, and zeroes dq_accum when it is set), bit 1
 // dK/dV kernel, bit 2 dQ kernel (the split backward).
 cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned mask);
