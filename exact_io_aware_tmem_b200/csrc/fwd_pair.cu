@@ -92,9 +92,9 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
   return __all_sync(FULL, ok);
 }
 
-// 320 threads x 200 registers fit the register file; the softmax threads hold
-// a whole 128-score row.
-__global__ void __maxnreg__(200)
+// 320 threads: ten warps, three on two of the four SM sub-partitions, whose
+// 16K registers then allow 168 per thread.
+__global__ void __launch_bounds__(THREADS, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m2,
@@ -327,16 +327,15 @@ __global__ void __maxnreg__(200)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= nvalid) r[c][i] = __float_as_uint(-INFINITY);
       }
-      // Row max with 8 independent partial maxima.
-      float mx8[8];
+      // Row max with 4 independent partial maxima.
+      float mx4[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+      for (int i = 0; i < 4; ++i) mx4[i] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(r[c][i]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(r[c][i]));
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_cand = mx * c2;
       const bool grow = m_cand > m_ref + RESCALE_LOG2;   // always true on the first visible tile
       const float m_new = grow ? m_cand : m_ref;
