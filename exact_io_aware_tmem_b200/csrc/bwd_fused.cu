@@ -78,12 +78,9 @@ struct Cfg {
   static_assert(D == 64 || D == 128, "head dim");
   static constexpr uint32_t TILE = BT * D * 2;       // one 128-row bf16 tile of Q, K, V or dO
   static constexpr int QS = 2;                       // Q stages (with LSE, D_i)
-  static constexpr int GS = 2;                       // dO stages
+  static constexpr int GS = 1;                       // dO stages (dO_{t+1} is read after dV_t)
   static constexpr bool ALIAS = D == 128;            // dQ_t formed over dP
-  // D = 128: the product is dQ_t^T = K^T dS^T, head dim on the TMEM lanes, so
-  // that one warp-wide add covers 32 consecutive head-dim entries of a query
-  // row: a whole 128-byte line of the accumulator per instruction.
-  static constexpr bool DQT = D == 128;
+  static constexpr int NBOX = D / 64;                // 32 x 32 fp32 dQ boxes per dS warp per step
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr uint32_t TM_DQ = ALIAS ? TM_DP : 256 + 2 * D;
   static constexpr uint32_t OFF_K = 0;
@@ -91,7 +88,8 @@ struct Cfg {
   static constexpr uint32_t OFF_Q = OFF_V + TILE;
   static constexpr uint32_t OFF_DO = OFF_Q + QS * TILE;
   static constexpr uint32_t OFF_DS = OFF_DO + GS * TILE;       // dS^T: 128 keys x 128 queries bf16
-  static constexpr uint32_t OFF_LSE = OFF_DS + 2 * SPAN;       // float [QS][BT]: LSE * log2(e)
+  static constexpr uint32_t OFF_STG = OFF_DS + 2 * SPAN;       // dQ staging: 4 KB per dS warp
+  static constexpr uint32_t OFF_LSE = OFF_STG + 8 * 4096;      // float [QS][BT]: LSE * log2(e)
   static constexpr uint32_t OFF_DLT = OFF_LSE + QS * BT * 4;   // float [QS][BT]: D_i
   static constexpr uint32_t OFF_BAR = OFF_DLT + QS * BT * 4;
   // kv_full, q_full[QS], q_empty[QS], do_full[GS], do_empty[GS], s_full,
@@ -161,20 +159,37 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
   }
 }
 
-// *dst += x (fp32, global, relaxed reduction at GPU scope; the accumulator is
-// only read by a later kernel).
-__device__ __forceinline__ void red_add(float* dst, float x) {
-  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(dst), "f"(x) : "memory");
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
 }
 
-// dst[0..31] += a[0..31], as above.
-__device__ __forceinline__ void red_add_row32(float* dst, const uint32_t (&a)[32]) {
-#pragma unroll
-  for (int v = 0; v < 8; ++v)
-    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * v),
-                 "f"(__uint_as_float(a[4 * v + 0])), "f"(__uint_as_float(a[4 * v + 1])),
-                 "f"(__uint_as_float(a[4 * v + 2])), "f"(__uint_as_float(a[4 * v + 3]))
-                 : "memory");
+// Global [y .. y + 31, x .. x + 31] (fp32) += the 32 x 32 box at ``src``
+// (128-byte swizzled), by the tensor-memory accelerator; completion is
+// tracked per issuing thread in bulk groups.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int x,
+                                                  int y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// This thread's bulk groups have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// This thread's bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 template <int D>
@@ -182,7 +197,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_do, const AttnParams p, int num_j,
+                     const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_dqa, const AttnParams p, int num_j,
                      int group) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -311,8 +327,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t leader = elect_one();
     constexpr uint32_t ID_SDP = idesc_bf16(BT, BT, false, false);  // S^T, dP^T
     constexpr uint32_t ID_KV = idesc_bf16(BT, D, false, true);     // dV, dK (A from TMEM)
-    constexpr uint32_t ID_DQ = C::DQT ? idesc_bf16(D, BT, true, true)    // dQ_t^T = K^T dS^T
-                                      : idesc_bf16(BT, D, true, true);   // dQ_t = dS K
+    constexpr uint32_t ID_DQ = idesc_bf16(BT, D, true, true);      // dQ_t = dS K
     const uint64_t k_kmaj = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
     const uint64_t v_kmaj = sdesc_sw128(sbase + C::OFF_V, 16, 1024);
     const uint64_t q_kmaj = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
@@ -388,14 +403,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
       }
 #pragma unroll
-      for (int kk = 0; kk < BT / 16; ++kk) {
-        // K-dim = 128 keys in steps of 16 (16 rows of both tiles).
-        const uint64_t ds = sdesc_add(ds_mn, kk * 2048), kt = sdesc_add(k_mn, kk * 2048);
-        if constexpr (C::DQT)
-          mma_ss_if(leader, tmem + C::TM_DQ, kt, ds, ID_DQ, kk > 0);
-        else
-          mma_ss_if(leader, tmem + C::TM_DQ, ds, kt, ID_DQ, kk > 0);
-      }
+      for (int kk = 0; kk < BT / 16; ++kk)   // K-dim = 128 keys in steps of 16
+        mma_ss_if(leader, tmem + C::TM_DQ, sdesc_add(ds_mn, kk * 2048), sdesc_add(k_mn, kk * 2048),
+                  ID_DQ, kk > 0);
       tc_commit_if(leader, bars.dq_full());
       if (more) {
         if (C::ALIAS) {
@@ -432,54 +442,45 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* ds_row = smem + C::OFF_DS + hf * SPAN + r * 128;
     float* const dq_acc = p.dq_accum;
 
-    // Adds the dQ partial of step tq (in TMEM) into dQacc.
+    // Adds the dQ partial of step tq (in TMEM) into dQacc. Thread = query row
+    // (warp & 3) * 32 + lane of the step's tile; the warp's 32 rows x 32
+    // columns form one box, staged 128-byte swizzled in shared memory and
+    // added by a TMA tensor reduction, which runs on its own while the warp
+    // goes on. At D = 128 the second box of a step is staged in this warp's
+    // 4 KB slice of the dS tile (free until dS of the next step, and written
+    // then only by this warp), the first in its slice of the staging area.
+    const uint32_t stg[2] = {sbase + C::OFF_STG + warp * 4096u, sbase + C::OFF_DS + warp * 4096u};
     auto drain_dq = [&](int tq) -> bool {
       if (!warp_wait(bars.dq_full(), tq & 1, p.err, abort, W_DQFULL)) return false;
       tc_fence_after();
-      constexpr int NC = C::DQT ? 2 : D / 64;   // 32-column blocks per thread
-      uint32_t a[NC][32];
+      uint32_t a[C::NBOX][32];
 #pragma unroll
-      for (int c = 0; c < NC; ++c)
-        tmem_ld32(tmem + lane_off + C::TM_DQ + hf * (32 * NC) + 32 * c, a[c]);
+      for (int c = 0; c < C::NBOX; ++c)
+        tmem_ld32(tmem + lane_off + C::TM_DQ + hf * (D / 2) + 32 * c, a[c]);
       tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < NC; ++c) reg_fence(a[c]);
+      for (int c = 0; c < C::NBOX; ++c) reg_fence(a[c]);
       tc_fence_before();
       mbar_arrive(bars.dq_free());
       const int h = hk * g + tq / n_qt;
-      const int qtile = (i0 + tq % n_qt) * BT;
-      if constexpr (C::DQT) {
-        // Thread = head-dim entry d (TMEM lane); columns = queries
-        // [64 hf, 64 hf + 64) of the tile. Query q's row of dQacc starts at
-        // ((start + q) H + h) D; the warp's 32 lanes are 32 consecutive d.
-        const int d = (warp & 3) * 32 + lane;
-        const int q0 = qtile + 64 * hf;
-        const size_t row_step = static_cast<size_t>(p.H) * D;
-        float* col = dq_acc + static_cast<size_t>(sq.start + q0) * row_step +
-                     static_cast<size_t>(h) * D + d;
-        const int nq = min(64, sq.len - q0);   // valid queries of this half (warp-uniform)
-        if (nq >= 64) {
+      const int row0 = sq.start + (i0 + tq % n_qt) * BT + (warp & 3) * 32;
+      // The staging slices' previous contents (a step back) must have been read.
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+      for (int c = 0; c < C::NBOX; ++c) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              red_add(col + (32 * c + i) * row_step, __uint_as_float(a[c][i]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (32 * c + i < nq) red_add(col + (32 * c + i) * row_step, __uint_as_float(a[c][i]));
-        }
-      } else {
-        // Thread = query row (TMEM lane), columns [hf D / 2, hf D / 2 + D / 2).
-        const int qpos = qtile + (warp & 3) * 32 + lane;
-        if (qpos < sq.len) {
-          float* dst = dq_acc + (static_cast<size_t>(sq.start + qpos) * p.H + h) * D + hf * (D / 2);
-#pragma unroll
-          for (int c = 0; c < NC; ++c) red_add_row32(dst + 32 * c, a[c]);
-        }
+        for (int m = 0; m < 8; ++m)
+          st_shared_v4(stg[c] + lane * 128 + ((m ^ (lane & 7)) << 4), a[c][4 * m], a[c][4 * m + 1],
+                       a[c][4 * m + 2], a[c][4 * m + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        // Rows past the sequence's end hold exact zeros (their dS rows are
+        // zero), so adding them to the next sequence's rows changes nothing;
+        // rows past the tensor are clipped by the copy.
+        if (lane == 0) tma_reduce_add_2d(&tm_dqa, stg[c], h * D + hf * (D / 2) + 32 * c, row0);
       }
+      if (lane == 0) bulk_commit();
       return true;
     };
 
@@ -550,8 +551,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // dS^T over the first 32 of this half's own 64 dP^T columns (A of dK),
-      // and into the shared dS^T tile (A of dQ, read MN-major).
+      // and into the shared dS^T tile (A of dQ, read MN-major). At D = 128
+      // this warp's slice of the tile staged a dQ box: its read must be done.
       tmem_st32(tmem + lane_off + C::TM_DP + 64 * hf, dsk);
+      if (C::NBOX > 1) {
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
 #pragma unroll
       for (int m = 0; m < 8; ++m)
         *reinterpret_cast<uint4*>(ds_row + ((m ^ (r & 7)) << 4)) =
@@ -562,6 +568,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(bars.ds_ready());
     }
     if (ok && n_steps > 0) ok = drain_dq(n_steps - 1);
+    // The reductions read this CTA's shared memory: all must be done before exit.
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
     // --------------------------------------------------- dK / dV epilogue ---
     if (ok && warp_wait(bars.dkv_done(), 0, p.err, abort, W_DKV)) {
       tc_fence_after();
@@ -624,6 +633,9 @@ cudaError_t launch_fused_d(const AttnParams& p, cudaStream_t stream) {
       !make_tmap_bf16_3d(&tv, p.v, p.total, p.H_kv, D, 1, fused::BT) ||
       !make_tmap_bf16_3d(&tg, p.dout, p.total, p.H, D, 1, fused::BT))
     return cudaErrorInvalidValue;
+  CUtensorMap ta;
+  if (!make_tmap_f32_2d(&ta, p.dq_accum, p.total, static_cast<unsigned long long>(p.H) * D, 32, 32))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fused::bwd_fused_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
@@ -631,7 +643,7 @@ cudaError_t launch_fused_d(const AttnParams& p, cudaStream_t stream) {
   // g query heads.
   const int group = l2_group(8ll * p.max_seqlen * D * (p.H / p.H_kv), 1, p.H_kv * p.B);
   fused::bwd_fused_kernel<D><<<static_cast<unsigned>(tiles), fused::THREADS, C::SMEM, stream>>>(
-      tq, tk, tv, tg, p, num_t, group);
+      tq, tk, tv, tg, ta, p, num_t, group);
   return cudaGetLastError();
 }
 

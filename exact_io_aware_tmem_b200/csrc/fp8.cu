@@ -20,14 +20,14 @@ namespace fa {
 namespace {
 
 constexpr int QBLOCK = 128;
-constexpr int QTHREADS = 256;
+constexpr int QTHREADS = 512;
 
 // One CTA per (sequence, head, 128-token block). Thread i holds the 8-element
-// groups i, i + 256, ... of the block in registers (PER groups at most), so
+// groups i, i + 512, ... of the block in registers (PER groups at most), so
 // the block is read from memory once: loaded, its max |x| reduced over the
 // CTA, then converted from the registers and written as codes.
 template <int PER>
-__global__ void __launch_bounds__(QTHREADS)
+__global__ void __launch_bounds__(QTHREADS, 2)
     fp8_quantize_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ x8,
                         float* __restrict__ scale, int N, int Hx, int D, int nb) {
   const int t = blockIdx.x % nb;
@@ -95,7 +95,7 @@ cudaError_t launch_fp8_quantize(const void* x, void* x8, float* scale, int B, in
   const long long blocks = static_cast<long long>(B) * Hx * nb;
   if (blocks == 0) return cudaSuccess;
   if (blocks > INT_MAX || D % 8 != 0 || D > 256) return cudaErrorInvalidValue;
-  // Groups of 8 per thread: ceil(128 rows * D / 8 / 256).
+  // Groups of 8 per thread: ceil(128 rows * D / 8 / 512).
   const int per = (QBLOCK * (D / 8) + QTHREADS - 1) / QTHREADS;
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   auto* q8 = static_cast<uint8_t*>(x8);
@@ -104,10 +104,8 @@ cudaError_t launch_fp8_quantize(const void* x, void* x8, float* scale, int B, in
     fp8_quantize_kernel<2><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
   else if (per <= 4)
     fp8_quantize_kernel<4><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
-  else if (per <= 8)
-    fp8_quantize_kernel<8><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
   else
-    fp8_quantize_kernel<16><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
+    fp8_quantize_kernel<8><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
   return cudaGetLastError();
 }
 

@@ -166,6 +166,10 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long long ro
 bool make_tmap_u8_2d(CUtensorMap* map, const void* base, unsigned long long rows,
                      unsigned long long cols, unsigned box_cols, unsigned box_rows);
 
+// Host: as make_tmap_bf16_2d for an fp32 tensor (box_cols fp32 columns).
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, unsigned long long rows,
+                      unsigned long long cols, unsigned box_cols, unsigned box_rows);
+
 // Host: 3-D bf16 view (D, heads, rows) of a token-major [rows, heads, D]
 // tensor with a (64, box_heads, box_rows) box and 128-byte swizzle. Column
 // blocks at x >= D lie outside the tensor and arrive as zeros.
