@@ -64,7 +64,11 @@ SIGNATURES = {
     "fa_fwd_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                            c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_void_p]),
     "fa_version": (c_int, []),
+    "fa_debug_build": (c_int, []),
+    "fa_debug_set_trace": (c_int, [c_void_p, c_size_t, c_int]),
 }
+DEBUG_TRACE_BYTES = 32 * 1024 * 8
+DEBUG_LIB_PATH = os.path.join(PKG, "libfa_b200_debug.so")
 
 _lib = None
 
@@ -78,21 +82,36 @@ class FAError(RuntimeError):
         super().__init__(f"{what}: {msg}")
 
 
+def _load(path: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m exact_io_aware_tmem_b200.build`"
+            " (the package has no non-CUDA fallback)")
+    handle = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
+
+
 def lib() -> ctypes.CDLL:
     """The loaded library (loaded once)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_tmem_b200.build`"
-                " (the package has no non-CUDA fallback)")
-        handle = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(handle, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = handle
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+_debug_lib = None
+
+
+def debug_lib() -> ctypes.CDLL:
+    """The debug build (index checks, event stamps); loaded once, on request."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _load(DEBUG_LIB_PATH)
+    return _debug_lib
 
 
 def check(status: int, what: str) -> None:

@@ -12,12 +12,30 @@ Layouts (token-major, as in include/fa.h):
 """
 from __future__ import annotations
 
+import contextlib
 import math
 from typing import Optional
 
 import torch
 
 from . import _abi
+
+# The library the entry points call: libfa_b200.so, or, inside debug_build(),
+# the same kernels built with index checks and event stamps.
+_lib = _abi.lib
+
+
+@contextlib.contextmanager
+def debug_build():
+    """Route the entry points through libfa_b200_debug.so (include/fa.h,
+    "Debug build") for the duration of the block."""
+    global _lib
+    prev = _lib
+    _lib = _abi.debug_lib
+    try:
+        yield _abi.debug_lib()
+    finally:
+        _lib = prev
 
 _DTYPES = {torch.bfloat16: _abi.FA_BF16, torch.float32: _abi.FA_F32}
 
@@ -66,7 +84,7 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = Fal
         lse = torch.empty((B, H, N) if cu_seqlens is None else (H, T), device=q.device,
                           dtype=torch.float32)
     s = -1.0 if scale is None else float(scale)
-    st = _abi.lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, N, D,
+    st = _lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, N, D,
                            _DTYPES[q.dtype], int(bool(causal)), s, _ptr(cu_seqlens), max_sl, T,
                            _stream(q.device))
     _abi.check(st, "fa_fwd")
@@ -79,7 +97,7 @@ BWD_SPLIT = _abi.BWD_SPLIT
 
 def workspace_size(T: int, H: int, D: int, dtype: torch.dtype, phases: int = BWD_FUSED) -> int:
     """Bytes of backward workspace for ``phases`` (fa_bwd_phases_workspace_size)."""
-    return int(_abi.lib().fa_bwd_phases_workspace_size(int(phases), T, H, D, _DTYPES[dtype]))
+    return int(_lib().fa_bwd_phases_workspace_size(int(phases), T, H, D, _DTYPES[dtype]))
 
 
 def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -107,7 +125,7 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     s = -1.0 if scale is None else float(scale)
-    st = _abi.lib().fa_bwd_phases(int(phases), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+    st = _lib().fa_bwd_phases(int(phases), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                   _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, H_kv, N, D,
                                   _DTYPES[q.dtype], int(bool(causal)), s, _ptr(cu_seqlens),
                                   max_sl, T, _ptr(workspace),
@@ -118,12 +136,12 @@ def bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
 
 def decode_num_splits(B: int, H_kv: int, max_seqlen_k: int, n_split: int = 0) -> int:
-    return int(_abi.lib().fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split))
+    return int(_lib().fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split))
 
 
 def decode_workspace_size(B: int, q_len: int, H: int, H_kv: int, D: int, max_seqlen_k: int,
                           n_split: int = 0) -> int:
-    return int(_abi.lib().fa_decode_workspace_size(B, q_len, H, H_kv, D, max_seqlen_k, n_split))
+    return int(_lib().fa_decode_workspace_size(B, q_len, H, H_kv, D, max_seqlen_k, n_split))
 
 
 def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -152,7 +170,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     need = decode_workspace_size(B, q_len, H, H_kv, D, max_seqlen_k, n_split)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
-    st = _abi.lib().fa_decode(
+    st = _lib().fa_decode(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), _ptr(cache_seqlens),
         _ptr(block_table), B, int(q_len), H, H_kv, D, int(page_size), int(max_blocks), rows,
         int(max_seqlen_k), int(causal), -1.0 if scale is None else float(scale), int(n_split),
@@ -169,7 +187,7 @@ def fp8_quantize(x: torch.Tensor, B: int, N: int, *, out: Optional[torch.Tensor]
     x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if out is None else out
     sc = torch.empty((B, Hx, (N + 127) // 128), dtype=torch.float32, device=x.device) \
         if scale is None else scale
-    st = _abi.lib().fa_fp8_quantize(_ptr(x), _ptr(x8), _ptr(sc), B, N, Hx, D, _stream(x.device))
+    st = _lib().fa_fp8_quantize(_ptr(x), _ptr(x8), _ptr(sc), B, N, Hx, D, _stream(x.device))
     _abi.check(st, "fa_fp8_quantize")
     return x8, sc
 
@@ -185,7 +203,7 @@ def fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v: torch.Tensor, q_scale: torch.
         out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
-    st = _abi.lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(q_scale), _ptr(k_scale),
+    st = _lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(q_scale), _ptr(k_scale),
                                _ptr(out), _ptr(lse), B, H, H_kv, N, D, int(bool(causal)),
                                -1.0 if scale is None else float(scale), _stream(q8.device))
     _abi.check(st, "fa_fwd_fp8")
@@ -197,18 +215,18 @@ def check_device_error(device: Optional[torch.device] = None) -> tuple:
     import ctypes
     dev = torch.device("cuda") if device is None else device
     where = ctypes.c_uint(0)
-    st = _abi.lib().fa_check_device_error(_stream(dev), ctypes.byref(where))
+    st = _lib().fa_check_device_error(_stream(dev), ctypes.byref(where))
     return st, where.value
 
 
 def selftest_wait_timeout(cycles: int, device: Optional[torch.device] = None) -> None:
     dev = torch.device("cuda") if device is None else device
-    _abi.check(_abi.lib().fa_selftest_wait_timeout(int(cycles), _stream(dev)),
+    _abi.check(_lib().fa_selftest_wait_timeout(int(cycles), _stream(dev)),
                "fa_selftest_wait_timeout")
 
 
 def set_wait_budget(cycles: int) -> None:
-    _abi.lib().fa_set_wait_budget(int(cycles))
+    _lib().fa_set_wait_budget(int(cycles))
 
 
 def default_scale(D: int) -> float:

@@ -121,6 +121,14 @@ struct Bars {
   __device__ uint32_t dkv_done() const { return b + 8u * (7 + 2 * C::QS + 2 * C::GS); }
 };
 
+// Event kinds of the debug build's stamps (one per step t unless noted).
+enum : int {
+  T_P_Q = 0, T_P_DO = 1, T_M_PREADY = 2, T_M_SNEXT = 3 /* S_{t+1}, index t+1 */,
+  T_M_DSREADY = 4, T_M_DQ = 5, T_M_DQFREE = 6, T_M_DP = 7 /* dP_{t+1}, index t+1 */,
+  T_S_SFULL = 8, T_S_PREADY = 9, T_S_DQFULL = 10, T_S_DQFREE = 11, T_S_STAGED = 12,
+  T_S_DPFULL = 13, T_S_DSREADY = 14, T_M_DV = 15
+};
+
 enum : unsigned {
   W_KV = 0x40100, W_QEMPTY = 0x40200, W_QFULL = 0x40300, W_SFULL = 0x40400, W_PREADY = 0x40500,
   W_DPFULL = 0x40600, W_DSREADY = 0x40700, W_DKV = 0x40800, W_DOFULL = 0x40900,
@@ -299,6 +307,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) {
         mbar_arrive_expect_tx(bars.q_full(st), C::TILE);
         load_tile<D>(sbase + C::OFF_Q + st * C::TILE, &tm_q, bars.q_full(st), h, row_q);
+        FA_STAMP(p, T_P_Q, t);
       }
 #pragma unroll
       for (int k = 0; k < BT / 32; ++k) {
@@ -311,6 +320,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) {
         mbar_arrive_expect_tx(bars.do_full(gt), C::TILE);
         load_tile<D>(sbase + C::OFF_DO + gt * C::TILE, &tm_do, bars.do_full(gt), h, row_q);
+        FA_STAMP(p, T_P_DO, t);
       }
       if (t + 1 < n_steps) fetch(t + 1);
     }
@@ -375,12 +385,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool more = t + 1 < n_steps;
       // dV += P^T_t dO_t (K-dim = 128 queries of the step).
       if (!(ok = warp_wait(bars.p_ready(), t & 1, p.err, abort, W_PREADY))) break;
+      if (lane == 0) FA_STAMP(p, T_M_PREADY, t);
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < BT / 16; ++kk)
         mma_ts_if(leader, tmem + C::TM_DV, tmem + C::TM_S + packed_col(kk),
                   sdesc_add(g_mn, gt * C::TILE + kk * 2048), ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
       tc_commit_if(leader, bars.do_empty(gt));
+      if (lane == 0) FA_STAMP(p, T_M_DV, t);
       // S^T_{t+1}: overwrites P^T_t, so it follows dV_t in the tensor pipe.
       if (more) {
         if (!(ok = warp_wait(bars.q_full((t + 1) % C::QS), ((t + 1) / C::QS) & 1, p.err, abort,
@@ -388,9 +400,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         tc_fence_after();
         issue_s((t + 1) % C::QS);
+        if (lane == 0) FA_STAMP(p, T_M_SNEXT, t + 1);
       }
       // dK += dS^T_t Q_t, then dQ_t = dS_t K (K-dim = 128 keys).
       if (!(ok = warp_wait(bars.ds_ready(), t & 1, p.err, abort, W_DSREADY))) break;
+      if (lane == 0) FA_STAMP(p, T_M_DSREADY, t);
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < BT / 16; ++kk)
@@ -407,16 +421,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         mma_ss_if(leader, tmem + C::TM_DQ, sdesc_add(ds_mn, kk * 2048), sdesc_add(k_mn, kk * 2048),
                   ID_DQ, kk > 0);
       tc_commit_if(leader, bars.dq_full());
+      if (lane == 0) FA_STAMP(p, T_M_DQ, t);
       if (more) {
         if (C::ALIAS) {
           // dP_{t+1} overwrites dQ_t: wait until it has been read out.
           if (!(ok = warp_wait(bars.dq_free(), t & 1, p.err, abort, W_DQFREE))) break;
+          if (lane == 0) FA_STAMP(p, T_M_DQFREE, t);
         }
         if (!(ok = warp_wait(bars.do_full((t + 1) % C::GS), ((t + 1) / C::GS) & 1, p.err, abort,
                              W_DOFULL)))
           break;
         tc_fence_after();
         issue_dp((t + 1) % C::GS);
+        if (lane == 0) FA_STAMP(p, T_M_DP, t + 1);
       }
     }
     tc_commit_if(leader, bars.dkv_done());
@@ -440,7 +457,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     // This thread's 128-byte row block of the dS^T tile (keys = rows, 64
     // queries per 128-byte block, 16-byte chunks XOR-swizzled by row & 7).
     uint8_t* ds_row = smem + C::OFF_DS + hf * SPAN + r * 128;
-    float* const dq_acc = p.dq_accum;
 
     // Adds the dQ partial of step tq (in TMEM) into dQacc. Thread = query row
     // (warp & 3) * 32 + lane of the step's tile; the warp's 32 rows x 32
@@ -450,8 +466,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // 4 KB slice of the dS tile (free until dS of the next step, and written
     // then only by this warp), the first in its slice of the staging area.
     const uint32_t stg[2] = {sbase + C::OFF_STG + warp * 4096u, sbase + C::OFF_DS + warp * 4096u};
+    const bool stamp = threadIdx.x == 0;   // debug stamps: lane 0 of warp 0
     auto drain_dq = [&](int tq) -> bool {
       if (!warp_wait(bars.dq_full(), tq & 1, p.err, abort, W_DQFULL)) return false;
+      if (stamp) FA_STAMP(p, T_S_DQFULL, tq);
       tc_fence_after();
       uint32_t a[C::NBOX][32];
 #pragma unroll
@@ -462,6 +480,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < C::NBOX; ++c) reg_fence(a[c]);
       tc_fence_before();
       mbar_arrive(bars.dq_free());
+      if (stamp) FA_STAMP(p, T_S_DQFREE, tq);
       const int h = hk * g + tq / n_qt;
       const int row0 = sq.start + (i0 + tq % n_qt) * BT + (warp & 3) * 32;
       // The staging slices' previous contents (a step back) must have been read.
@@ -478,9 +497,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         // Rows past the sequence's end hold exact zeros (their dS rows are
         // zero), so adding them to the next sequence's rows changes nothing;
         // rows past the tensor are clipped by the copy.
-        if (lane == 0) tma_reduce_add_2d(&tm_dqa, stg[c], h * D + hf * (D / 2) + 32 * c, row0);
+        if (lane == 0 && FA_CHECK(p, row0 >= 0 && row0 < p.total && h < p.H, 0xDB0402u))
+          tma_reduce_add_2d(&tm_dqa, stg[c], h * D + hf * (D / 2) + 32 * c, row0);
       }
       if (lane == 0) bulk_commit();
+      if (stamp) FA_STAMP(p, T_S_STAGED, tq);
       return true;
     };
 
@@ -492,6 +513,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float* dlt_t = s_dlt + st * BT + 64 * hf;
       if (!(ok = warp_wait(bars.q_full(st), (t / C::QS) & 1, p.err, abort, W_QFULL))) break;
       if (!(ok = warp_wait(bars.s_full(), t & 1, p.err, abort, W_SFULL))) break;
+      if (stamp) FA_STAMP(p, T_S_SFULL, t);
       tc_fence_after();
       const bool full = qbase >= qlo && qbase + 64 <= qhi;
       uint32_t pk[32];   // P^T as packed bf16, the value dS is formed from
@@ -523,11 +545,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bars.p_ready());
+      if (stamp) FA_STAMP(p, T_S_PREADY, t);
 
       // dQ of the previous step: its product ran under this step's exponentials.
       if (t > 0 && !(ok = drain_dq(t - 1))) break;
 
       if (!(ok = warp_wait(bars.dp_full(), t & 1, p.err, abort, W_DPFULL))) break;
+      if (stamp) FA_STAMP(p, T_S_DPFULL, t);
       tc_fence_after();
       uint32_t dsk[32];
 #pragma unroll
@@ -566,6 +590,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bars.ds_ready());
+      if (stamp) FA_STAMP(p, T_S_DSREADY, t);
     }
     if (ok && n_steps > 0) ok = drain_dq(n_steps - 1);
     // The reductions read this CTA's shared memory: all must be done before exit.
@@ -584,7 +609,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld_wait();
         reg_fence(a);
         reg_fence(v);
-        if (key_ok) {
+        if (key_ok && FA_CHECK(p, sq.start + kpos < p.total && hk < p.H_kv, 0xDB0401u)) {
           store_row_bf16(static_cast<__nv_bfloat16*>(p.dk) + off + 32 * c, a, p.scale);
           store_row_bf16(static_cast<__nv_bfloat16*>(p.dv) + off + 32 * c, v, 1.f);
         }

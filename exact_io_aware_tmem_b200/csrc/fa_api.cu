@@ -30,6 +30,10 @@ fa_status cuda_status(cudaError_t e) {
 }
 long long g_budget = kDefaultBudget;
 
+// Debug builds: the stamp buffer and traced CTA of the next launches.
+unsigned long long* g_trace = nullptr;
+int g_trace_cta = 0;
+
 constexpr int kMaxDevices = 64;
 unsigned* g_err_ptr[kMaxDevices] = {};
 std::mutex g_mu;
@@ -106,6 +110,8 @@ fa_status check_common(AttnParams& p, int B, int H, int H_kv, int N, int D, fa_d
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err.word = nullptr;
   p.err.budget = g_budget;
+  p.trace = g_trace;
+  p.trace_cta = g_trace_cta;
   return FA_OK;
 }
 
@@ -483,6 +489,34 @@ fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream) {
 }
 
 const char* fa_last_cuda_error_string(void) { return cudaGetErrorString(fa::g_last_cuda); }
+
+fa_status fa_debug_set_trace(void* buffer, size_t bytes, int cta) {
+#ifdef FA_DEBUG
+  if (buffer == nullptr) {
+    fa::g_trace = nullptr;
+    return FA_OK;
+  }
+  if (bytes < static_cast<size_t>(FA_DEBUG_TRACE_BYTES) || cta < 0 ||
+      (reinterpret_cast<uintptr_t>(buffer) & 7u) != 0)
+    return FA_ERR_INVALID_ARG;
+  fa::g_trace = static_cast<unsigned long long*>(buffer);
+  fa::g_trace_cta = cta;
+  return FA_OK;
+#else
+  (void)buffer;
+  (void)bytes;
+  (void)cta;
+  return FA_ERR_UNSUPPORTED;
+#endif
+}
+
+int fa_debug_build(void) {
+#ifdef FA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 int fa_version(void) { return 100; }
 

@@ -81,6 +81,14 @@ struct Bars {
   __device__ uint32_t o_full() const { return b + 8u * (5 + 2 * KS + 2 * VS); }
 };
 
+// Event kinds of the debug build's stamps (one per key tile j unless noted);
+// group g's softmax kinds are T_W_SFULL + 4 g, ...
+enum : int {
+  T_P_K = 0, T_P_V = 1, T_M_VFULL = 2, T_M_PV0 = 3, T_M_S0 = 4 /* S_0 of tile j+1, index j+1 */,
+  T_M_PV1 = 5, T_M_S1 = 6 /* index j+1 */, T_W_SFULL = 7, T_W_LD = 8, T_W_EXP = 9, T_W_ARR = 10,
+  T_M_PREADY0 = 15, T_M_PREADY1 = 16
+};
+
 enum : unsigned {
   W_Q = 0x50100, W_KEMPTY = 0x50200, W_VEMPTY = 0x50300, W_KFULL = 0x50400, W_VFULL = 0x50500,
   W_SFULL = 0x50600, W_PREADY = 0x50700, W_OFULL = 0x50800, BAD_ALIGN = 0x50900
@@ -184,6 +192,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int c = 0; c < 2; ++c)
             tma_load_2d(sbase + OFF_K + st * TILE + c * SPAN, &tm_k, bars.k_full(st),
                         hk * D + c * 64, sq.start + jk * BN);
+          FA_STAMP(p, T_P_K, jk);
         }
         __syncwarp();
         ++jk;
@@ -197,6 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int c = 0; c < 2; ++c)
             tma_load_2d(sbase + OFF_V + st * TILE + c * SPAN, &tm_v, bars.v_full(st),
                         hk * D + c * 64, sq.start + jv * BN);
+          FA_STAMP(p, T_P_V, jv);
         }
         __syncwarp();
         ++jv;
@@ -267,6 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int j = 0; ok && j < n_kv; ++j) {
       if (!(ok = warp_wait(bars.v_full(j % VS), (j / VS) & 1, p.err, abort, W_VFULL))) break;
+      if (lane == 0) FA_STAMP(p, T_M_VFULL, j);
       const bool next = j + 1 < n_kv;
       bool k_next = false;   // K_{j+1} seen in shared memory
 #pragma unroll
@@ -274,8 +285,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int n_g = g ? n_1 : n_0;
         if (j < n_g) {
           if (!(ok = warp_wait(bars.p_ready(g), j & 1, p.err, abort, W_PREADY))) break;
+          if (lane == 0) FA_STAMP(p, g ? T_M_PREADY1 : T_M_PREADY0, j);
           tc_fence_after();
           issue_pv(g, j);
+          if (lane == 0) FA_STAMP(p, g ? T_M_PV1 : T_M_PV0, j);
         }
         // S_g of the next tile overwrites P_g: it follows P_g V_j.
         if (j + 1 < n_g) {
@@ -287,6 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             k_next = true;
           }
           issue_s(g, j + 1);
+          if (lane == 0) FA_STAMP(p, g ? T_M_S1 : T_M_S0, j + 1);
         }
       }
       if (!ok) break;
@@ -307,11 +321,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t o_col = tmem + lane_off + TM_O + g * D;
     const float c2 = p.scale_log2;
     const int n = g ? n_1 : n_0;
+    const bool stamp = quarter == 0 && lane == 0;   // debug stamps: first warp of each group
+    [[maybe_unused]] const int tk = 4 * g;
     float m_ref = -INFINITY;  // reference max (log2 units)
     float l = 0.f;            // row sum in that reference
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
       if (!(ok = warp_wait(bars.s_full(g), j & 1, p.err, abort, W_SFULL))) break;
+      if (stamp) FA_STAMP(p, T_W_SFULL + tk, j);
       tc_fence_after();
       uint32_t r[4][32];
 #pragma unroll
@@ -319,6 +336,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+      if (stamp) FA_STAMP(p, T_W_LD + tk, j);
       const int nvalid = lim - j * BN + 1;   // visible keys in this tile
       if (nvalid < BN) {
 #pragma unroll
@@ -356,6 +374,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_st16(s_col + 16 * c, pk);
       }
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      if (stamp) FA_STAMP(p, T_W_EXP + tk, j);
       // The reference moved: rescale the row sum and (from the second tile
       // on) the O row, which holds P V of the earlier tiles only: S_g of this
       // tile completing means P_g V of the previous tile has completed.
@@ -377,6 +396,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bars.p_ready(g));
+      if (stamp) FA_STAMP(p, T_W_ARR + tk, j);
     }
     // ------------------------------------------------------------ epilogue ---
     if (ok && n > 0 && warp_wait(bars.o_full(), 0, p.err, abort, W_OFULL)) {
@@ -389,7 +409,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(o_col + 32 * c, o);
         tmem_ld_wait();
         reg_fence(o);
-        if (row_ok) {
+        if (row_ok && FA_CHECK(p, out_row < static_cast<size_t>(p.total) * p.H, 0xDB0501u)) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + out_row * D +
                                                 32 * c);
 #pragma unroll

@@ -30,7 +30,36 @@ struct AttnParams {
   float scale;      // multiplies Q K^T
   float scale_log2; // scale * log2(e)
   DevErr err;
+  // Debug builds (FA_DEBUG): where one CTA records the clock of its events,
+  // or null. [kinds][1024] 64-bit stamps; see FA_STAMP.
+  unsigned long long* trace;
+  int trace_cta;
 };
+
+// Debug builds only: stamp event ``kind`` of step ``idx`` with the SM clock,
+// in the traced CTA. The caller picks one thread per event (lane 0 of the
+// role's warp). Compiled out otherwise.
+#ifdef FA_DEBUG
+#define FA_STAMP(p, kind, idx)                                                       \
+  do {                                                                               \
+    if ((p).trace != nullptr && static_cast<int>(blockIdx.x) == (p).trace_cta &&     \
+        (idx) >= 0 && (idx) < 1024)                                                  \
+      (p).trace[(kind) * 1024 + (idx)] = static_cast<unsigned long long>(clock64()); \
+  } while (0)
+// Debug builds only: a failed index check is recorded in the device error
+// word (ERR_BOUNDS, ``where``) and the access is skipped by the caller.
+#define FA_CHECK(p, cond, where) ((cond) ? true : (fa::record_bounds_dbg((p).err, (where)), false))
+#else
+#define FA_STAMP(p, kind, idx) \
+  do {                         \
+  } while (0)
+#define FA_CHECK(p, cond, where) true
+#endif
+
+__device__ __forceinline__ void record_bounds_dbg(const DevErr& e, unsigned where) {
+  atomicOr(e.word, ERR_BOUNDS);
+  atomicExch(e.word + 1, where);
+}
 
 struct SeqInfo {
   int start;

@@ -1,0 +1,169 @@
+"""Event timelines of one CTA, recorded by the debug build of the library.
+
+The debug build (``python -m exact_io_aware_tmem_b200.build --debug``,
+libfa_b200_debug.so) stamps the SM clock at the events of each role of the
+traced CTA: waits passed, products issued, signals sent, one stamp per step
+(include/fa.h, "Debug build"). This module runs one pass of a kernel on a
+workload through that build and reports, over the steady-state steps, the
+median number of cycles between the events: where each role waits, and for
+what.
+
+  python -m exact_io_aware_tmem_b200.trace --kernel bwd --workload NAME [--cta 0]
+  python -m exact_io_aware_tmem_b200.trace --kernel fwd --workload NAME
+
+The traced CTA is blockIdx.x (0: the first launched, with the longest causal
+work).
+"""
+from __future__ import annotations
+
+import argparse
+import statistics
+import sys
+
+# Event kinds, as numbered in the kernels' sources.
+BWD_KINDS = {
+    "P_Q": 0, "P_DO": 1, "M_PREADY": 2, "M_SNEXT": 3, "M_DSREADY": 4, "M_DQ": 5,
+    "M_DQFREE": 6, "M_DP": 7, "S_SFULL": 8, "S_PREADY": 9, "S_DQFULL": 10, "S_DQFREE": 11,
+    "S_STAGED": 12, "S_DPFULL": 13, "S_DSREADY": 14, "M_DV": 15,
+}
+FWD_KINDS = {
+    "P_K": 0, "P_V": 1, "M_VFULL": 2, "M_PV0": 3, "M_S0": 4, "M_PV1": 5, "M_S1": 6,
+    "W0_SFULL": 7, "W0_LD": 8, "W0_EXP": 9, "W0_ARR": 10,
+    "W1_SFULL": 11, "W1_LD": 12, "W1_EXP": 13, "W1_ARR": 14,
+    "M_PREADY0": 15, "M_PREADY1": 16,
+}
+# (label, from event, step offset of from, to event, step offset of to): the
+# median of stamp[to][t + dto] - stamp[from][t + dfrom] over the steps t.
+BWD_SPANS = [
+    ("dS warps: exponentials of S_t (s_full -> p_ready)", "S_SFULL", 0, "S_PREADY", 0),
+    ("dS warps: wait for dQ_{t-1} (p_ready -> dq_full)", "S_PREADY", 0, "S_DQFULL", -1),
+    ("dS warps: read dQ_{t-1} out of TMEM", "S_DQFULL", -1, "S_DQFREE", -1),
+    ("dS warps: stage dQ_{t-1}, issue reductions", "S_DQFREE", -1, "S_STAGED", -1),
+    ("dS warps: wait for dP_t (-> dp_full)", "S_STAGED", -1, "S_DPFULL", 0),
+    ("dS warps: dS phase (dp_full -> ds_ready)", "S_DPFULL", 0, "S_DSREADY", 0),
+    ("dS warps: wait for S_{t+1} (ds_ready -> s_full)", "S_DSREADY", 0, "S_SFULL", 1),
+    ("step period (s_full -> s_full)", "S_SFULL", 0, "S_SFULL", 1),
+    ("MMA: p_ready seen after arrival", "S_PREADY", 0, "M_PREADY", 0),
+    ("MMA: dV_t issued (p_ready seen -> issued)", "M_PREADY", 0, "M_DV", 0),
+    ("MMA: S_{t+1} issued after dV_t", "M_DV", 0, "M_SNEXT", 1),
+    ("MMA: ds_ready seen after arrival", "S_DSREADY", 0, "M_DSREADY", 0),
+    ("MMA: dK_t, dQ_t issued (ds_ready seen -> dQ issued)", "M_DSREADY", 0, "M_DQ", 0),
+    ("MMA: dq_free seen after arrival", "S_DQFREE", 0, "M_DQFREE", 0),
+    ("MMA: dP_{t+1} issued after dq_free", "M_DQFREE", 0, "M_DP", 1),
+    ("tensor: S_{t+1} issue -> s_full seen", "M_SNEXT", 1, "S_SFULL", 1),
+    ("tensor: dQ_t issue -> dq_full seen", "M_DQ", 0, "S_DQFULL", 0),
+    ("tensor: dP_{t+1} issue -> dp_full seen", "M_DP", 1, "S_DPFULL", 1),
+    ("producer: Q_{t+1} issued before S_{t+1} issue", "P_Q", 1, "M_SNEXT", 1),
+    ("producer: dO_{t+1} issued before dP_{t+1} issue", "P_DO", 1, "M_DP", 1),
+]
+FWD_SPANS = [
+    ("group 0: load S (s_full -> scores in registers)", "W0_SFULL", 0, "W0_LD", 0),
+    ("group 0: max, exponentials, P stored (-> exp done)", "W0_LD", 0, "W0_EXP", 0),
+    ("group 0: rescale, P visible (-> p_ready)", "W0_EXP", 0, "W0_ARR", 0),
+    ("group 0: wait for next scores (p_ready -> s_full)", "W0_ARR", 0, "W0_SFULL", 1),
+    ("group 0: tile period", "W0_SFULL", 0, "W0_SFULL", 1),
+    ("group 1: load S", "W1_SFULL", 0, "W1_LD", 0),
+    ("group 1: max, exponentials, P stored", "W1_LD", 0, "W1_EXP", 0),
+    ("group 1: rescale, P visible", "W1_EXP", 0, "W1_ARR", 0),
+    ("group 1: wait for next scores", "W1_ARR", 0, "W1_SFULL", 1),
+    ("group 1: tile period", "W1_SFULL", 0, "W1_SFULL", 1),
+    ("group 1 start after group 0 start", "W0_SFULL", 0, "W1_SFULL", 0),
+    ("MMA: p_ready(0) seen after arrival", "W0_ARR", 0, "M_PREADY0", 0),
+    ("MMA: P_0 V_j issued", "M_PREADY0", 0, "M_PV0", 0),
+    ("MMA: S_0 of j+1 issued after P_0 V_j", "M_PV0", 0, "M_S0", 1),
+    ("MMA: p_ready(1) seen after arrival", "W1_ARR", 0, "M_PREADY1", 0),
+    ("MMA: wait for p_ready(1) after S_0 issue", "M_S0", 1, "M_PREADY1", 0),
+    ("tensor: S_0 issue -> s_full seen by group 0", "M_S0", 1, "W0_SFULL", 1),
+    ("tensor: S_1 issue -> s_full seen by group 1", "M_S1", 1, "W1_SFULL", 1),
+    ("producer: K_{j+1} issued before S_0 of j+1 issue", "P_K", 1, "M_S0", 1),
+    ("producer: V_j issued before the MMA saw it", "P_V", 0, "M_VFULL", 0),
+]
+
+
+def spans(stamps, kinds: dict, table, n_steps: int, skip: int = 2) -> list:
+    """(label, median cycles, count) for each span of ``table``."""
+    out = []
+    for label, a, da, b, db in table:
+        d = []
+        for t in range(skip, n_steps - skip):
+            ta, tb = t + da, t + db
+            if not (0 <= ta < 1024 and 0 <= tb < 1024):
+                continue
+            x, y = int(stamps[kinds[a]][ta]), int(stamps[kinds[b]][tb])
+            if x and y:
+                d.append(y - x)
+        out.append((label, statistics.median(d) if d else None, len(d)))
+    return out
+
+
+def run(kernel: str, workload: str, cta: int = 0):
+    """Runs the forward (and, for ``bwd``, the backward) of the workload on
+    cuda:0 through the debug build with stamping on for the kernel asked
+    for. Returns (stamps [32, 1024] int64 numpy, steps of the traced CTA)."""
+    import torch
+
+    from . import attention as fa
+    from . import _abi
+    from .workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS[workload]
+    inp = make_inputs(w)
+    B = len(inp.cu_seqlens) - 1
+    dev = torch.device("cuda", 0)
+
+    def to_dev(t):
+        t = t.to(dev)
+        return t if inp.varlen else t.view(B, w.N, t.shape[1], w.D)
+
+    q, k, v, do = (to_dev(t) for t in (inp.q, inp.k, inp.v, inp.do))
+    kw = dict(causal=w.causal, scale=w.scale)
+    if inp.varlen:
+        kw.update(cu_seqlens=inp.cu_seqlens.to(dev), max_seqlen=inp.max_seqlen)
+    buf = torch.zeros(_abi.DEBUG_TRACE_BYTES // 8, dtype=torch.int64, device=dev)
+    with fa.debug_build() as lib:
+        assert lib.fa_debug_build() == 1
+        if kernel == "fwd":
+            _abi.check(lib.fa_debug_set_trace(buf.data_ptr(), buf.numel() * 8, cta), "trace")
+            o, lse = fa.fwd(q, k, v, **kw)
+            _abi.check(lib.fa_debug_set_trace(None, 0, 0), "trace")
+        else:
+            o, lse = fa.fwd(q, k, v, **kw)
+            T = q.numel() // (w.H * w.D)
+            ws = torch.empty(fa.workspace_size(T, w.H, w.D, q.dtype), dtype=torch.uint8,
+                             device=dev)
+            fa.bwd(do, q, k, v, o, lse, workspace=ws, phases=_abi.BWD_PREPROCESS, **kw)
+            _abi.check(lib.fa_debug_set_trace(buf.data_ptr(), buf.numel() * 8, cta), "trace")
+            fa.bwd(do, q, k, v, o, lse, workspace=ws, phases=_abi.BWD_FUSED_KERNEL, **kw)
+            _abi.check(lib.fa_debug_set_trace(None, 0, 0), "trace")
+            fa.bwd(do, q, k, v, o, lse, workspace=ws, phases=_abi.BWD_DQ_CONVERT, **kw)
+        st, where = fa.check_device_error(dev)
+        if st != 0:
+            raise RuntimeError(f"device error {st} at {where:#x}")
+    stamps = buf.view(32, 1024).cpu().numpy()
+    # Steps of the traced CTA: query steps (backward) or key tiles (forward;
+    # the second query tile of a causal pair has one more than the first).
+    firsts = ["S_SFULL"] if kernel == "bwd" else ["W0_SFULL", "W1_SFULL"]
+    kinds = BWD_KINDS if kernel == "bwd" else FWD_KINDS
+    n = max(int((stamps[kinds[f]] != 0).sum()) for f in firsts)
+    return stamps, n
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--kernel", choices=["fwd", "bwd"], required=True)
+    ap.add_argument("--workload", default="bf16_causal_b2_h16_n8192_d128")
+    ap.add_argument("--cta", type=int, default=0)
+    args = ap.parse_args(argv)
+    from .build import build
+    build(debug=True)
+    stamps, n = run(args.kernel, args.workload, args.cta)
+    kinds, table = (BWD_KINDS, BWD_SPANS) if args.kernel == "bwd" else (FWD_KINDS, FWD_SPANS)
+    print(f"{args.kernel} {args.workload} CTA {args.cta}: {n} steps stamped; median cycles "
+          f"over the steady-state steps")
+    for label, med, cnt in spans(stamps, kinds, table, n):
+        print(f"  {label:62s} {'-' if med is None else f'{med:8.0f}'}  ({cnt})")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

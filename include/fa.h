@@ -266,6 +266,29 @@ void fa_set_wait_budget(long long cycles);
 fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream);
 
 /*
+ * Debug build. The library built with -DFA_DEBUG (libfa_b200_debug.so, same
+ * entry points) checks indices in its kernels against the buffers they
+ * address, recording a failed check in the device error word
+ * (fa_check_device_error reports FA_ERR_INVALID_ARG, ``where`` names the
+ * check) and skipping the access, and can record, for one CTA of each launch,
+ * the SM clock at the events of its roles (waits passed, products issued,
+ * signals sent): per kind of event, one 64-bit stamp per step.
+ *
+ * fa_debug_build - 1 in the debug build, 0 otherwise.
+ *
+ * fa_debug_set_trace - launches enqueued after the call stamp their events
+ * into ``buffer`` (device memory of at least FA_DEBUG_TRACE_BYTES, 8-byte
+ * aligned, owned by the caller: [32 kinds][1024 steps] unsigned 64-bit
+ * clocks, entries of events that did not happen left as they were) for the
+ * CTA with blockIdx.x == ``cta``. A null buffer stops stamping. The kinds of
+ * each kernel are listed in exact_io_aware_tmem_b200/trace.py. Returns
+ * FA_ERR_UNSUPPORTED in the ordinary build.
+ */
+#define FA_DEBUG_TRACE_BYTES (32u * 1024u * 8u)
+int fa_debug_build(void);
+fa_status fa_debug_set_trace(void* buffer, size_t bytes, int cta);
+
+/*
  * ---------------------------------------------------------------- decode ---
  * Split-KV decode (FlashDecoding) over a contiguous or paged key/value cache.
  *

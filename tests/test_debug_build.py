@@ -1,0 +1,90 @@
+"""The debug build (libfa_b200_debug.so): the same kernels with index checks
+that record into the device error word instead of trapping, and per-role
+event stamps of one CTA (include/fa.h, "Debug build").
+
+The GPU tests run small causal and packed cases through it, check them against
+the float64 oracle with the parity tolerances, check that no index check
+fired, and that the stamps of a traced CTA form a timeline.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_tmem_b200 as fa
+from exact_io_aware_tmem_b200 import _abi
+from exact_io_aware_tmem_b200 import attention as fa_att
+from exact_io_aware_tmem_b200 import trace
+from exact_io_aware_tmem_b200.workloads import random_case
+from oracle import attention as oa
+from tests._util import f64, o_excess_bf16, rel_fro, to_api
+
+
+@pytest.fixture(scope="module")
+def debug_lib():
+    from exact_io_aware_tmem_b200 import build
+    build.build()
+    build.build(debug=True)
+    return _abi.debug_lib()
+
+
+def test_debug_build_loads_and_reports_itself(debug_lib):
+    assert debug_lib.fa_debug_build() == 1
+    assert _abi.lib().fa_debug_build() == 0
+    # The ordinary build records no stamps.
+    assert _abi.lib().fa_debug_set_trace(ctypes.c_void_p(256), _abi.DEBUG_TRACE_BYTES, 0) == \
+        _abi.FA_ERR_UNSUPPORTED
+    # Argument checks of the debug build's trace switch (no device access).
+    assert debug_lib.fa_debug_set_trace(ctypes.c_void_p(256), 8, 0) == _abi.FA_ERR_INVALID_ARG
+    assert debug_lib.fa_debug_set_trace(ctypes.c_void_p(256), _abi.DEBUG_TRACE_BYTES, -1) == \
+        _abi.FA_ERR_INVALID_ARG
+    assert debug_lib.fa_debug_set_trace(None, 0, 0) == _abi.FA_OK
+
+
+CASES = [
+    # (lengths, H, H_kv, D, varlen, causal)
+    ([384, 384], 4, 2, 128, False, True),
+    ([5, 0, 128, 1, 300, 129, 64], 4, 2, 128, True, False),
+    ([300, 129, 257], 4, 4, 64, True, True),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("lengths,H,H_kv,D,varlen,causal", CASES)
+def test_debug_build_parity_and_clean_checks(debug_lib, lengths, H, H_kv, D, varlen, causal):
+    inp = random_case(31, dtype="bf16", lengths=lengths, H=H, H_kv=H_kv, D=D, varlen=varlen)
+    B = len(lengths)
+    N = 0 if varlen else lengths[0]
+    a = to_api(inp, B, N)
+    kw = dict(causal=causal, cu_seqlens=a.get("cu_seqlens"), max_seqlen=a.get("max_seqlen"))
+    with fa_att.debug_build():
+        o, lse = fa.fwd(a["q"], a["k"], a["v"], **kw)
+        grads = fa.bwd(a["do"], a["q"], a["k"], a["v"], o, lse, **kw)
+        st, where = fa.check_device_error()
+    assert st == 0, f"debug build reported {st} at {where:#x}"
+    scale = D ** -0.5
+    ro, _ = oa.attention_forward(inp.q, inp.k, inp.v, inp.cu_seqlens.numpy(), causal, scale)
+    T = inp.q.shape[0]
+    assert o_excess_bf16(f64(o).reshape(T, H, D), ro) <= 0
+    ref = oa.attention_backward(inp.q, inp.k, inp.v, inp.do, inp.cu_seqlens.numpy(), causal, scale)
+    for g, r in zip(grads, ref):
+        assert rel_fro(f64(g).reshape(r.shape), r) <= 3e-2
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("kernel", ["fwd", "bwd"])
+def test_debug_build_stamps_form_a_timeline(debug_lib, kernel):
+    """One traced CTA of the causal B2 H16 N8192 workload: every step of the
+    traced roles is stamped, in order."""
+    stamps, n = trace.run(kernel, "bf16_causal_b2_h16_n8192_d128", cta=0)
+    kinds = trace.BWD_KINDS if kernel == "bwd" else trace.FWD_KINDS
+    first = "S_SFULL" if kernel == "bwd" else "W1_SFULL"
+    # CTA 0 is the longest causal one: 64 key tiles (forward, second query
+    # tile of the last pair) or 64 query tiles (backward, key tile 0).
+    assert n == 64
+    s = stamps[kinds[first]][:n].astype(np.int64)
+    assert (np.diff(s) > 0).all()
+    table = trace.BWD_SPANS if kernel == "bwd" else trace.FWD_SPANS
+    for label, med, cnt in trace.spans(stamps, kinds, table, n):
+        assert med is not None and cnt > 0, label
