@@ -56,19 +56,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// How long (ns) a waiting thread may be suspended before it re-checks its
+// phase (0: no hint, plain try_wait).
+#ifndef FA_SUSPEND_NS
+#define FA_SUSPEND_NS 2000
+#endif
+
 // As mbar_try_wait, but a thread whose phase is not complete yet may be
-// suspended (up to about 2 microseconds) until it completes, instead of
-// spinning and taking issue slots from the warps doing the work.
+// suspended (up to FA_SUSPEND_NS) until it completes, instead of spinning and
+// taking issue slots from the warps doing the work.
 __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+#if FA_SUSPEND_NS > 0
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "n"(2000)
+      : "r"(bar), "r"(parity), "n"(FA_SUSPEND_NS)
       : "memory");
   return ok != 0;
+#else
+  return mbar_try_wait(bar, parity);
+#endif
 }
 
 // Wait until the phase of ``bar`` with the given parity has completed. Gives
