@@ -496,8 +496,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         // Rows past the sequence's end hold exact zeros (their dS rows are
         // zero), so adding them to the next sequence's rows changes nothing;
-        // rows past the tensor are clipped by the copy.
-        if (lane == 0 && FA_CHECK(p, row0 >= 0 && row0 < p.total && h < p.H, 0xDB0402u))
+        // rows past the tensor are clipped by the copy. A box wholly past the
+        // sequence is not added at all.
+        if (lane == 0 && row0 < sq.start + sq.len &&
+            FA_CHECK(p, row0 >= 0 && row0 < p.total && h < p.H, 0xDB0402u))
           tma_reduce_add_2d(&tm_dqa, stg[c], h * D + hf * (D / 2) + 32 * c, row0);
       }
       if (lane == 0) bulk_commit();

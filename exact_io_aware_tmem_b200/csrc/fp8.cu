@@ -20,14 +20,10 @@ namespace fa {
 namespace {
 
 constexpr int QBLOCK = 128;
-constexpr int QTHREADS = 512;
+constexpr int QTHREADS = 256;
 
-// One CTA per (sequence, head, 128-token block). Thread i holds the 8-element
-// groups i, i + 512, ... of the block in registers (PER groups at most), so
-// the block is read from memory once: loaded, its max |x| reduced over the
-// CTA, then converted from the registers and written as codes.
-template <int PER>
-__global__ void __launch_bounds__(QTHREADS, 2)
+// One CTA per (sequence, head, 128-token block); 8 elements per step.
+__global__ void __launch_bounds__(QTHREADS)
     fp8_quantize_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ x8,
                         float* __restrict__ scale, int N, int Hx, int D, int nb) {
   const int t = blockIdx.x % nb;
@@ -43,17 +39,14 @@ __global__ void __launch_bounds__(QTHREADS, 2)
     return (static_cast<size_t>(b) * N + r0 + row) * Hx * D + static_cast<size_t>(h) * D +
            (i % per_row) * 8;
   };
-  uint4 v[PER];
   float amax = 0.f;
+  for (int i = threadIdx.x; i < n; i += QTHREADS) {
+    const uint4 v = *reinterpret_cast<const uint4*>(x + offset(i));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int i = threadIdx.x + k * QTHREADS;
-    v[k] = (i < n) ? __ldg(reinterpret_cast<const uint4*>(x + offset(i))) : make_uint4(0, 0, 0, 0);
-    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      amax = fmaxf(amax, fabsf(__uint_as_float(w[e] << 16)));
-      amax = fmaxf(amax, fabsf(__uint_as_float(w[e] & 0xffff0000u)));
+    for (int k = 0; k < 4; ++k) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[k] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(w[k] & 0xffff0000u)));
     }
   }
   __shared__ float red[QTHREADS / 32];
@@ -66,24 +59,20 @@ __global__ void __launch_bounds__(QTHREADS, 2)
   for (int k = 1; k < QTHREADS / 32; ++k) amax = fmaxf(amax, red[k]);
   const float delta = (amax > 0.f) ? __fdiv_rn(amax, 448.f) : 1.f;
   if (threadIdx.x == 0) scale[static_cast<size_t>(bh) * nb + t] = delta;
+  for (int i = threadIdx.x; i < n; i += QTHREADS) {
+    const size_t o = offset(i);
+    const uint4 v = *reinterpret_cast<const uint4*>(x + o);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed[2];
 #pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int i = threadIdx.x + k * QTHREADS;
-    if (i < n) {
-      const uint32_t lo = pack_e4m3x2(__fdiv_rn(__uint_as_float(v[k].x << 16), delta),
-                                      __fdiv_rn(__uint_as_float(v[k].x & 0xffff0000u), delta)) |
-                          (static_cast<uint32_t>(pack_e4m3x2(
-                               __fdiv_rn(__uint_as_float(v[k].y << 16), delta),
-                               __fdiv_rn(__uint_as_float(v[k].y & 0xffff0000u), delta)))
-                           << 16);
-      const uint32_t hi = pack_e4m3x2(__fdiv_rn(__uint_as_float(v[k].z << 16), delta),
-                                      __fdiv_rn(__uint_as_float(v[k].z & 0xffff0000u), delta)) |
-                          (static_cast<uint32_t>(pack_e4m3x2(
-                               __fdiv_rn(__uint_as_float(v[k].w << 16), delta),
-                               __fdiv_rn(__uint_as_float(v[k].w & 0xffff0000u), delta)))
-                           << 16);
-      *reinterpret_cast<uint2*>(x8 + offset(i)) = make_uint2(lo, hi);
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t a = pack_e4m3x2(__fdiv_rn(__uint_as_float(w[2 * k] << 16), delta),
+                                     __fdiv_rn(__uint_as_float(w[2 * k] & 0xffff0000u), delta));
+      const uint32_t c = pack_e4m3x2(__fdiv_rn(__uint_as_float(w[2 * k + 1] << 16), delta),
+                                     __fdiv_rn(__uint_as_float(w[2 * k + 1] & 0xffff0000u), delta));
+      packed[k] = a | (c << 16);
     }
+    *reinterpret_cast<uint2*>(x8 + o) = make_uint2(packed[0], packed[1]);
   }
 }
 
@@ -94,18 +83,9 @@ cudaError_t launch_fp8_quantize(const void* x, void* x8, float* scale, int B, in
   const int nb = (N + QBLOCK - 1) / QBLOCK;
   const long long blocks = static_cast<long long>(B) * Hx * nb;
   if (blocks == 0) return cudaSuccess;
-  if (blocks > INT_MAX || D % 8 != 0 || D > 256) return cudaErrorInvalidValue;
-  // Groups of 8 per thread: ceil(128 rows * D / 8 / 512).
-  const int per = (QBLOCK * (D / 8) + QTHREADS - 1) / QTHREADS;
-  const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  auto* q8 = static_cast<uint8_t*>(x8);
-  const unsigned g = static_cast<unsigned>(blocks);
-  if (per <= 2)
-    fp8_quantize_kernel<2><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
-  else if (per <= 4)
-    fp8_quantize_kernel<4><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
-  else
-    fp8_quantize_kernel<8><<<g, QTHREADS, 0, stream>>>(xb, q8, scale, N, Hx, D, nb);
+  if (blocks > INT_MAX || D % 8 != 0) return cudaErrorInvalidValue;
+  fp8_quantize_kernel<<<static_cast<unsigned>(blocks), QTHREADS, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(x8), scale, N, Hx, D, nb);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,5 @@
-// Attention forward at D = 128, two 128-row query tiles per CTA, bf16 in /
-// fp32 accumulate, on the sm_100a tensor cores.
+// Attention forward, two 128-row query tiles per CTA, bf16 in / fp32
+// accumulate, on the sm_100a tensor cores (D = 64 and 128).
 //
 // What it computes: for every query row, the online-softmax recurrence of
 // aiqz.cc "Flash Attention V2/V3 optimization", section "V2 algorithm
@@ -26,7 +26,7 @@
 //               S_1 = Q_1 K_{j+1}^T, so each group exponentiates tile j+1
 //               while the tensor core works for the other group.
 // The two groups share nothing but the K / V tiles: each owns its S, P and O
-// in TMEM (S_g [128 g, 128 g + 128), O_g [256 + 128 g, ...), P_g as bf16 over
+// in TMEM (S_g [128 g, 128 g + 128), O_g [256 + D g, ...), P_g as bf16 over
 // the first 64 columns of S_g once the scores are in registers). S_g of tile
 // j+1 completing implies P_g V_j has completed (the tensor core runs one
 // thread's MMAs in order and a commit covers all earlier ones), so a group
@@ -41,7 +41,6 @@ namespace {
 
 namespace pair {
 
-constexpr int D = 128;
 constexpr int BM = 128;            // rows per query tile
 constexpr int BN = 128;            // keys per tile
 constexpr int THREADS = 320;
@@ -49,23 +48,31 @@ constexpr int WARP_TMA = 8;
 constexpr int WARP_MMA = 9;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S = 0;       // S_g at TM_S + 128 g
-constexpr uint32_t TM_O = 256;     // O_g at TM_O + 128 g
+constexpr uint32_t TM_O = 256;     // O_g at TM_O + D g
 constexpr uint32_t SPAN = 128 * 128;          // 128 rows x 128 bytes (one swizzle column block)
-constexpr uint32_t TILE = BM * D * 2;         // 32 KB
-constexpr int KS = 3;              // K stages
-constexpr int VS = 2;              // V stages
-constexpr uint32_t OFF_Q = 0;                 // Q_0, Q_1
-constexpr uint32_t OFF_K = OFF_Q + 2 * TILE;
-constexpr uint32_t OFF_V = OFF_K + KS * TILE;
-constexpr uint32_t OFF_BAR = OFF_V + VS * TILE;
-// q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2],
-// p_ready[2], o_full
-constexpr int NBAR = 1 + 2 * KS + 2 * VS + 5;
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-// No alignment slack: the dynamic shared memory must start on a 1024-byte
-// boundary (128-byte swizzle atoms); the kernel checks and reports.
-constexpr uint32_t SMEM = OFF_MISC + 16;
-static_assert(SMEM <= 232448, "shared memory budget");
+constexpr int KS_MAX = 4;
+constexpr int VS_MAX = 4;
+
+template <int D>
+struct Cfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr uint32_t TILE = BM * D * 2;       // 32 KB at D = 128
+  static constexpr int KS = D == 128 ? 3 : 4;        // K stages
+  static constexpr int VS = D == 128 ? 2 : 4;        // V stages
+  static constexpr uint32_t OFF_Q = 0;               // Q_0, Q_1
+  static constexpr uint32_t OFF_K = OFF_Q + 2 * TILE;
+  static constexpr uint32_t OFF_V = OFF_K + KS * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_V + VS * TILE;
+  // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2],
+  // p_ready[2], o_full (laid out for the largest ring depths)
+  static constexpr int NBAR = 1 + 2 * KS_MAX + 2 * VS_MAX + 5;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  // No alignment slack: the dynamic shared memory must start on a 1024-byte
+  // boundary (128-byte swizzle atoms); the kernel checks and reports.
+  static constexpr uint32_t SMEM = OFF_MISC + 16;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(KS <= KS_MAX && VS <= VS_MAX, "ring depths");
+};
 constexpr float RESCALE_LOG2 = 8.f;
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -73,12 +80,12 @@ struct Bars {
   uint32_t b;
   __device__ uint32_t q_full() const { return b; }
   __device__ uint32_t k_full(int s) const { return b + 8u * (1 + s); }
-  __device__ uint32_t k_empty(int s) const { return b + 8u * (1 + KS + s); }
-  __device__ uint32_t v_full(int s) const { return b + 8u * (1 + 2 * KS + s); }
-  __device__ uint32_t v_empty(int s) const { return b + 8u * (1 + 2 * KS + VS + s); }
-  __device__ uint32_t s_full(int g) const { return b + 8u * (1 + 2 * KS + 2 * VS + g); }
-  __device__ uint32_t p_ready(int g) const { return b + 8u * (3 + 2 * KS + 2 * VS + g); }
-  __device__ uint32_t o_full() const { return b + 8u * (5 + 2 * KS + 2 * VS); }
+  __device__ uint32_t k_empty(int s) const { return b + 8u * (1 + KS_MAX + s); }
+  __device__ uint32_t v_full(int s) const { return b + 8u * (1 + 2 * KS_MAX + s); }
+  __device__ uint32_t v_empty(int s) const { return b + 8u * (1 + 2 * KS_MAX + VS_MAX + s); }
+  __device__ uint32_t s_full(int g) const { return b + 8u * (1 + 2 * KS_MAX + 2 * VS_MAX + g); }
+  __device__ uint32_t p_ready(int g) const { return b + 8u * (3 + 2 * KS_MAX + 2 * VS_MAX + g); }
+  __device__ uint32_t o_full() const { return b + 8u * (5 + 2 * KS_MAX + 2 * VS_MAX); }
 };
 
 // Event kinds of the debug build's stamps (one per key tile j unless noted);
@@ -102,11 +109,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
 
 // 320 threads: ten warps, three on two of the four SM sub-partitions, whose
 // 16K registers then allow 168 per thread.
+template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m2,
                     int group) {
+  using C = Cfg<D>;
+  constexpr int KS = C::KS, VS = C::VS;
+  constexpr uint32_t TILE = C::TILE, OFF_Q = C::OFF_Q, OFF_K = C::OFF_K, OFF_V = C::OFF_V;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if ((sbase & 1023u) != 0) {
@@ -132,9 +143,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int n_1 = ((2 * m2 + 1) * BM >= sq.len) ? 0 : (p.causal ? min(n_all, 2 * m2 + 2) : n_all);
   const int n_kv = max(n_0, n_1);
 
-  const Bars bars{sbase + OFF_BAR};
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  const Bars bars{sbase + C::OFF_BAR};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
@@ -176,7 +187,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // never written out).
       mbar_arrive_expect_tx(bars.q_full(), 2 * TILE);
       for (int g = 0; g < 2; ++g)
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < D / 64; ++c)
           tma_load_2d(sbase + OFF_Q + g * TILE + c * SPAN, &tm_q, bars.q_full(), h * D + c * 64,
                       sq.start + (2 * m2 + g) * BM);
     }
@@ -189,7 +200,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int st = jk % KS;
         if (lane == 0) {
           mbar_arrive_expect_tx(bars.k_full(st), TILE);
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < D / 64; ++c)
             tma_load_2d(sbase + OFF_K + st * TILE + c * SPAN, &tm_k, bars.k_full(st),
                         hk * D + c * 64, sq.start + jk * BN);
           FA_STAMP(p, T_P_K, jk);
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int st = jv % VS;
         if (lane == 0) {
           mbar_arrive_expect_tx(bars.v_full(st), TILE);
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < D / 64; ++c)
             tma_load_2d(sbase + OFF_V + st * TILE + c * SPAN, &tm_v, bars.v_full(st),
                         hk * D + c * 64, sq.start + jv * BN);
           FA_STAMP(p, T_P_V, jv);
@@ -441,9 +452,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_fwd_pair(const AttnParams& p, cudaStream_t stream) {
+namespace {
+
+template <int D>
+cudaError_t launch_pair_d(const AttnParams& p, cudaStream_t stream) {
   using namespace pair;
-  if (p.D != D) return cudaErrorInvalidValue;
+  using C = Cfg<D>;
   const int num_m2 = (p.max_seqlen + 2 * BM - 1) / (2 * BM);
   const long long tiles = static_cast<long long>(num_m2) * p.H * p.B;
   if (tiles == 0 || p.total == 0) return cudaSuccess;
@@ -453,13 +467,21 @@ cudaError_t launch_fwd_pair(const AttnParams& p, cudaStream_t stream) {
       !make_tmap_bf16_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN) ||
       !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
     return cudaErrorInvalidValue;
-  cudaError_t e =
-      cudaFuncSetAttribute(fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t e = cudaFuncSetAttribute(fwd_pair_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int group = l2_group(4ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_pair_kernel<<<static_cast<unsigned>(tiles), THREADS, SMEM, stream>>>(tq, tk, tv, p, num_m2,
-                                                                           group);
+  fwd_pair_kernel<D><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(tq, tk, tv, p,
+                                                                                 num_m2, group);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_pair(const AttnParams& p, cudaStream_t stream) {
+  if (p.D == 64) return launch_pair_d<64>(p, stream);
+  if (p.D == 128) return launch_pair_d<128>(p, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace fa
