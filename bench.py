@@ -123,6 +123,7 @@ def source_sha(*names) -> str:
 
 
 KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "fwd_pair_kernel": ("fwd_pair.cu", "common.cuh", "params.h"),
                   "bwd_fused_kernel": ("bwd_fused.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
@@ -226,10 +227,11 @@ def oracle_sample(w, n_tokens: int):
     do = inp.do[:, 0].to(torch.float64).numpy()
     t0 = time.perf_counter()
     oa.head_forward(q, k, v, w.scale, w.causal)
-    oa.head_backward(q, k, v, do, w.scale, w.causal)
+    if w.backward:
+        oa.head_backward(q, k, v, do, w.scale, w.causal)
     dt = time.perf_counter() - t0
     fwd, bwd = step_flops([n_tokens], 1, w.D, w.causal)
-    return dt, fwd + bwd
+    return dt, fwd + (bwd if w.backward else 0.0)
 
 
 def oracle_tokens_for(w, seconds: float) -> int:
@@ -246,7 +248,7 @@ def cpu_baseline(w, seconds: float = 15.0) -> dict:
     dt, fl = oracle_sample(w, n)
     return {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "seconds": round(dt, 3),
-            "sample": f"float64 numpy oracle, forward+backward of one query head of "
+            "sample": f"float64 numpy oracle, {config_of(w)['pass']} of one query head of "
                       f"{w.name} truncated to N={n} (causal={w.causal}, D={w.D}); FLOPs by the "
                       f"same formula as the GPU line"}
 
@@ -266,7 +268,7 @@ def run_reference(args, w) -> None:
         tot_f += fl
     value = tot_f / tot_t / 1e12
     sample = (f"float64 numpy oracle, one query head of {w.name} truncated to N={n}, "
-              f"forward+backward per step")
+              f"{config_of(w)['pass']} per step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
@@ -282,7 +284,8 @@ def run_reference(args, w) -> None:
 def config_of(w) -> dict:
     from exact_io_aware_tmem_b200.workloads import make_inputs  # noqa: F401
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "D": w.D,
-            "causal": w.causal, "varlen": w.varlen is not None, "pass": "fwd+bwd",
+            "causal": w.causal, "varlen": w.varlen is not None,
+            "pass": "fwd+bwd" if w.backward else "fwd",
             "seed": w.seed}
 
 
@@ -380,7 +383,12 @@ def run_ours(args, w) -> None:
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.workspace_size(T, w.H, w.D, q.dtype), dtype=torch.uint8, device=dev)
     ph = fa.BWD_FUSED  # preprocess (+ accumulator zeroing), fused kernel, dQ conversion
-    bytes_in = sum(t.numel() * t.element_size() for t in (q, k, v, do))
+    # Forward-only workloads (the B4 N2048 D64 configuration) time the
+    # forward alone: their step is one fa_fwd.
+    do_bwd = w.backward
+    ins = (q, k, v, do) if do_bwd else (q, k, v)
+    bytes_in = sum(t.numel() * t.element_size() for t in ins)
+    fwd_name = "fwd_pair_kernel" if w.D == 128 else "fwd_bf16_kernel"
 
     def step(ev=None):
         if ev is not None:
@@ -388,6 +396,8 @@ def run_ours(args, w) -> None:
         fa.fwd(q, k, v, out=o, lse=lse, **kw)
         if ev is not None:
             ev[1].record()
+        if not do_bwd:
+            return
         fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph & 0x01, **kw)
         if ev is not None:
             ev[2].record()
@@ -431,27 +441,31 @@ def run_ours(args, w) -> None:
         raise RuntimeError(f"device error {st} at {where:#x} in the timed region")
     elapsed_ms = start.elapsed_time(end)
     max_ms = reduce_max(elapsed_ms, dev)
+    spans = {fwd_name: (0, 1)}
+    if do_bwd:
+        spans.update({"bwd_preprocess": (1, 2), "bwd_fused_kernel": (2, 3), "dq_convert": (3, 4)})
     k_ms = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
-            for name, (a, b) in {"fwd_bf16_kernel": (0, 1), "bwd_preprocess": (1, 2),
-                                 "bwd_fused_kernel": (2, 3), "dq_convert": (3, 4)}.items()}
+            for name, (a, b) in spans.items()}
     k_ms = {n: reduce_max(t, dev) for n, t in k_ms.items()}
 
     # End to end through the public API with host buffers: pinned H2D of the
     # step's inputs, forward + backward, D2H of every output, pipelined.
     e2e_steps = max(3, min(args.steps, 20))
-    host_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
-    outs = [o, lse, dq, dk, dv]
+    host_in = [t.cpu().pin_memory() for t in ins]
+    outs = [o, lse, dq, dk, dv] if do_bwd else [o, lse]
     bytes_out = sum(t.numel() * t.element_size() for t in outs)
 
-    def e2e_step(ins, outs_):
-        qq, kk, vv, dd = ins
-        oo, ll, gq, gk, gv = outs_
-        fa.fwd(qq, kk, vv, out=oo, lse=ll, **kw)
-        fa.bwd(dd, qq, kk, vv, oo, ll, workspace=ws, dq=gq, dk=gk, dv=gv, **kw)
+    def e2e_step(ins_, outs_):
+        qq, kk, vv = ins_[:3]
+        fa.fwd(qq, kk, vv, out=outs_[0], lse=outs_[1], **kw)
+        if do_bwd:
+            gq, gk, gv = outs_[2:]
+            fa.bwd(ins_[3], qq, kk, vv, outs_[0], outs_[1], workspace=ws, dq=gq, dk=gk, dv=gv,
+                   **kw)
 
     if world > 1:
         dist.barrier()
-    e2e_ms = reduce_max(pipelined_e2e(torch, dev, host_in, [q, k, v, do], outs, e2e_step,
+    e2e_ms = reduce_max(pipelined_e2e(torch, dev, host_in, list(ins), outs, e2e_step,
                                       e2e_steps), dev)
 
     if world > 1:
@@ -460,16 +474,22 @@ def run_ours(args, w) -> None:
     if rank != 0:
         return
 
+    if not do_bwd:
+        bwd_fl = 0.0
     per_step_fl = fwd_fl + bwd_fl
     value = aggregate(per_step_fl * args.steps, world, [max_ms / 1e3]) / 1e12
-    fwd_tf = fwd_fl / (k_ms["fwd_bf16_kernel"] / 1e3) / 1e12
-    bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_fused_kernel"] + k_ms["dq_convert"]
-    bwd_tf = bwd_fl / (bwd_ms / 1e3) / 1e12
+    fwd_tf = fwd_fl / (k_ms[fwd_name] / 1e3) / 1e12
+    bwd_tf = None
+    if do_bwd:
+        bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_fused_kernel"] + k_ms["dq_convert"]
+        bwd_tf = bwd_fl / (bwd_ms / 1e3) / 1e12
     # Dominant kernel: the one with the largest share of the step. Algorithmic
     # FLOPs per launch: the forward's two products (4 N^2 D per head) and the
     # fused backward's five (S, dP, dV, dK, dQ: 10 N^2 D, the method's 2.5x),
     # causal halving each.
-    kernel_fl = {"fwd_bf16_kernel": fwd_fl, "bwd_fused_kernel": bwd_fl}
+    kernel_fl = {fwd_name: fwd_fl}
+    if do_bwd:
+        kernel_fl["bwd_fused_kernel"] = bwd_fl
     dom = max(kernel_fl, key=lambda n: k_ms[n])
     dom_fl = kernel_fl[dom]
     achieved = dom_fl / (k_ms[dom] / 1e3) / 1e12
@@ -484,7 +504,7 @@ def run_ours(args, w) -> None:
                        ranks="each rank its own seeded batch of this shape"),
         "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
         "fwd_frac_of_peak": fwd_tf / peak,
-        "bwd_frac_of_peak": bwd_tf / peak,
+        "bwd_frac_of_peak": None if bwd_tf is None else bwd_tf / peak,
         "peak_tflops": {"burst": peaks["bf16_tflops"], "sustained": peaks["bf16_tflops_sustained"],
                         "source": peaks["source"]},
         "kernel_ms": {n: round(t, 4) for n, t in k_ms.items()},
@@ -501,7 +521,7 @@ def run_ours(args, w) -> None:
                 "d2h_bytes_per_step": bytes_out,
                 "how": "public API, pinned host buffers, copies of neighbouring steps "
                        "overlapping the computation (double-buffered, three streams)"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (4 if do_bwd else 1) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
