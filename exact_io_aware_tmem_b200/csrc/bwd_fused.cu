@@ -14,43 +14,41 @@
 // shared memory while the CTA walks the 128-row query tiles of every query
 // head of its GQA group (step t = one query tile of one head). Keys sit on the
 // TMEM lanes for the key-side products; per step, five products, each once:
-//     S^T  = K Q_t^T            (A, B in shared memory)         -> TMEM S
-//     dP^T = V dO_t^T           (A, B in shared memory)         -> TMEM dP
-//     dV  += P^T dO_t           (A = P^T, bf16 in TMEM over S)  -> TMEM dV
-//     dK  += dS^T Q_t           (A = dS^T, bf16 in TMEM over dP) -> TMEM dK
-//     dQ_t^T = K^T dS^T         (D = 128; A = K^T and B = dS^T read MN-major
-//                                from the K tile and from a swizzled dS^T
-//                                tile the dS warps also write to shared
-//                                memory; head dim on the TMEM lanes)
-//     dQ_t = dS K               (D = 64; the same tiles, queries on the lanes)
+//     S^T  = K Q_t^T            (A, B in shared memory)          -> TMEM S
+//     dP^T = V dO_t^T           (A, B in shared memory)          -> TMEM dP
+//     dV  += P^T dO_t           (A = P^T, bf16 in TMEM over S)   -> TMEM dV
+//     dQ_t = dS K               (A = dS, read MN-major from a swizzled dS^T
+//                                tile the dS warps write to shared memory;
+//                                queries on the TMEM lanes)      -> TMEM dQ
+//     dK  += dS^T Q_t           (A = dS^T, the same tile read K-major)
+//                                                                -> TMEM dK
 // and the fp32 dQ_t partial is added into the caller's fp32 accumulator
 // dQacc [T, H, D] (zeroed by the preprocess kernel; a convert kernel writes
-// dQ = bf16(scale dQacc) afterwards). With the head dim on the lanes, one
-// warp-wide reduction for one query covers 32 consecutive entries of its
-// accumulator row (a whole 128-byte line): at 64 KB of partials per step, the
-// line-per-instruction form is what keeps the additions at the L2's rate
-// (about twice that of one 16-byte piece of a different row per lane). The
-// accumulation order over key tiles is not fixed, so dQ is reproducible only
-// to rounding; dK and dV are summed in a fixed order inside one CTA.
+// dQ = bf16(scale dQacc) afterwards): each dS warp stages its 32 x 32 box of
+// dQ_t in shared memory and one lane adds it with a TMA tensor reduction,
+// which runs on its own while the warp goes on. The accumulation order over
+// key tiles is not fixed, so dQ is reproducible only to rounding; dK and dV
+// are summed in a fixed order inside one CTA.
 //
 // TMEM columns: S [0,128), dP [128,256), dV, dK after them. At D = 128 the
-// 512 columns are full, so dQ_t is formed over dP once dK_t has read dS^T
-// from there, and dP_{t+1} waits until the dS warps have read dQ_t out. At
-// D = 64 dQ_t has columns of its own.
+// 512 columns are full, so dQ_t is formed over dP (the dS warps have read dP_t
+// before they signal dS_t), and dP_{t+1} waits until they have read dQ_t out.
+// At D = 64 dQ_t has columns of its own.
 //
 // Roles (320 threads):
 //   warps 0-7  dS warps. Thread = key row (TMEM lane) for S^T / dP^T, warps w
 //              and w+4 taking query columns [64 hf, 64 hf + 64). Per step:
 //              exponentials of S^T_t -> P^T_t into TMEM; then the read-out of
-//              dQ_{t-1} (thread = head-dim entry at D = 128, query row at
-//              D = 64) and its addition into dQacc;
-//              then dS^T_t into TMEM and into the shared dS tile.
+//              dQ_{t-1} (thread = query row), staged for its reduction; then
+//              dS^T_t into the shared dS tile.
 //   warp 8     TMA producer: K, V once; Q_t (with the step's LSE and D_i
-//              staged beside it) and dO_t through two-stage rings.
+//              staged beside it) through a two-stage ring, dO_t through one
+//              stage (dV_t, its last reader, runs long before dP_{t+1}).
 //   warp 9     MMA warp, converged, one elect.sync lane issuing. Order per
-//              step: dV_t, S_{t+1}, dK_t, dQ_t, dP_{t+1}: the exponentials of
-//              step t+1 overlap dK_t and dQ_t, and the dS phase of step t
-//              overlaps dV_t and S_{t+1}.
+//              step: dP_t, dV_t, S_{t+1}, dQ_t, dK_t. dQ_t goes right after dS_t
+//              because its read-out gates dP_{t+1}; the exponentials of step
+//              t+1 overlap dQ_t and dK_t, and the dS phase of step t overlaps
+//              dV_t and S_{t+1}.
 #include <limits.h>
 #include <math.h>
 
@@ -93,8 +91,8 @@ struct Cfg {
   static constexpr uint32_t OFF_DLT = OFF_LSE + QS * BT * 4;   // float [QS][BT]: D_i
   static constexpr uint32_t OFF_BAR = OFF_DLT + QS * BT * 4;
   // kv_full, q_full[QS], q_empty[QS], do_full[GS], do_empty[GS], s_full,
-  // dp_full, p_ready, ds_ready, dq_full, dq_free, dkv_done
-  static constexpr int NBAR = 1 + 2 * QS + 2 * GS + 7;
+  // dp_full, p_ready, ds_ready, dq_full, dq_free, dkv_done, ds_free
+  static constexpr int NBAR = 1 + 2 * QS + 2 * GS + 8;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   // No alignment slack: the dynamic shared memory must start on a 1024-byte
   // boundary (128-byte swizzle atoms); the kernel checks and reports.
@@ -119,6 +117,8 @@ struct Bars {
   __device__ uint32_t dq_full() const { return b + 8u * (5 + 2 * C::QS + 2 * C::GS); }
   __device__ uint32_t dq_free() const { return b + 8u * (6 + 2 * C::QS + 2 * C::GS); }
   __device__ uint32_t dkv_done() const { return b + 8u * (7 + 2 * C::QS + 2 * C::GS); }
+  // dK_t has read the shared dS^T tile (which then takes a staged dQ box).
+  __device__ uint32_t ds_free() const { return b + 8u * (8 + 2 * C::QS + 2 * C::GS); }
 };
 
 // Event kinds of the debug build's stamps (one per step t unless noted).
@@ -126,13 +126,16 @@ enum : int {
   T_P_Q = 0, T_P_DO = 1, T_M_PREADY = 2, T_M_SNEXT = 3 /* S_{t+1}, index t+1 */,
   T_M_DSREADY = 4, T_M_DQ = 5, T_M_DQFREE = 6, T_M_DP = 7 /* dP_{t+1}, index t+1 */,
   T_S_SFULL = 8, T_S_PREADY = 9, T_S_DQFULL = 10, T_S_DQFREE = 11, T_S_STAGED = 12,
-  T_S_DPFULL = 13, T_S_DSREADY = 14, T_M_DV = 15
+  T_S_DPFULL = 13, T_S_DSREADY = 14, T_M_DV = 15, T_S_SLD = 16 /* scores in registers */,
+  T_S_EXPD = 17 /* exponentials done */, T_S_DPLD = 18 /* dP in registers */,
+  T_S_DSC = 19 /* dS formed */, T_S_DSST = 20 /* dS stored to shared memory */
 };
 
 enum : unsigned {
   W_KV = 0x40100, W_QEMPTY = 0x40200, W_QFULL = 0x40300, W_SFULL = 0x40400, W_PREADY = 0x40500,
   W_DPFULL = 0x40600, W_DSREADY = 0x40700, W_DKV = 0x40800, W_DOFULL = 0x40900,
-  W_DOEMPTY = 0x40A00, W_DQFULL = 0x40B00, W_DQFREE = 0x40C00, BAD_ALIGN = 0x40D00
+  W_DOEMPTY = 0x40A00, W_DQFULL = 0x40B00, W_DQFREE = 0x40C00, BAD_ALIGN = 0x40D00,
+  W_DSFREE = 0x40E00
 };
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DevErr& e,
@@ -258,6 +261,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bars.dq_full(), 1);
     mbar_init(bars.dq_free(), N_DS);
     mbar_init(bars.dkv_done(), 1);
+    mbar_init(bars.ds_free(), 1);
     fence_mbar_init();
   }
   if (warp == WARP_MMA) {
@@ -348,6 +352,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // dS as the A operand of dQ_t: queries (M) run along the rows of the dS^T
     // tile, in two 64-query column blocks one span apart; keys (K) down them.
     const uint64_t ds_mn = sdesc_sw128(sbase + C::OFF_DS, SPAN, 1024);
+    // dS^T as the A operand of dK: keys (M) down the rows, queries (K) along
+    // them, K-major like the Q and K tiles.
+    const uint64_t ds_kmaj = sdesc_sw128(sbase + C::OFF_DS, 16, 1024);
     auto issue_s = [&](int st) {     // S^T = K Q^T, K-dim = D
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -402,15 +409,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         issue_s((t + 1) % C::QS);
         if (lane == 0) FA_STAMP(p, T_M_SNEXT, t + 1);
       }
-      // dK += dS^T_t Q_t, then dQ_t = dS_t K (K-dim = 128 keys).
+      // dQ_t = dS_t K (K-dim = 128 keys), then dK += dS^T_t Q_t (K-dim = 128
+      // queries). Both read dS from the shared dS^T tile (MN-major for dQ,
+      // K-major for dK), so dQ_t - whose read-out gates dP_{t+1} - goes first.
       if (!(ok = warp_wait(bars.ds_ready(), t & 1, p.err, abort, W_DSREADY))) break;
       if (lane == 0) FA_STAMP(p, T_M_DSREADY, t);
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < BT / 16; ++kk)
-        mma_ts_if(leader, tmem + C::TM_DK, tmem + C::TM_DP + packed_col(kk),
-                  sdesc_add(q_mn, st * C::TILE + kk * 2048), ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
-      tc_commit_if(leader, bars.q_empty(st));
       if (!C::ALIAS && t > 0) {
         // dQ_{t-1} must have been read out of its columns.
         if (!(ok = warp_wait(bars.dq_free(), (t - 1) & 1, p.err, abort, W_DQFREE))) break;
@@ -422,6 +426,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                   ID_DQ, kk > 0);
       tc_commit_if(leader, bars.dq_full());
       if (lane == 0) FA_STAMP(p, T_M_DQ, t);
+#pragma unroll
+      for (int kk = 0; kk < BT / 16; ++kk) {
+        const uint32_t o = (kk >> 2) * SPAN + (kk & 3) * 32;   // queries 16 kk .. 16 kk + 15
+        mma_ss_if(leader, tmem + C::TM_DK, sdesc_add(ds_kmaj, o),
+                  sdesc_add(q_mn, st * C::TILE + kk * 2048), ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
+      }
+      tc_commit_if(leader, bars.q_empty(st));
+      tc_commit_if(leader, bars.ds_free());
       if (more) {
         if (C::ALIAS) {
           // dP_{t+1} overwrites dQ_t: wait until it has been read out.
@@ -486,6 +498,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // The staging slices' previous contents (a step back) must have been read.
       if (lane == 0) bulk_wait_read_all();
       __syncwarp();
+      // The second box goes into this warp's slice of the dS^T tile: dK_tq
+      // must have finished reading it.
+      if (C::NBOX > 1 && !warp_wait(bars.ds_free(), tq & 1, p.err, abort, W_DSFREE)) return false;
 #pragma unroll
       for (int c = 0; c < C::NBOX; ++c) {
 #pragma unroll
@@ -525,6 +540,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(tmem + lane_off + C::TM_S + 64 * hf + 32 * c, sr);
         tmem_ld_wait();
         reg_fence(sr);
+        if (stamp && c == 0) FA_STAMP(p, T_S_SLD, t);
         // LSE read four at a time (one broadcast load per four columns).
         const float4* lse4 = reinterpret_cast<const float4*>(lse_t + 32 * c);
 #pragma unroll
@@ -542,6 +558,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           pk[16 * c + (q >> 1)] = pack_bf16x2(p0, p1);
         }
       }
+      if (stamp) FA_STAMP(p, T_S_EXPD, t);
       // P^T over the first 32 of this half's own 64 S^T columns.
       tmem_st32(tmem + lane_off + C::TM_S + 64 * hf, pk);
       tmem_st_wait();
@@ -562,6 +579,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(tmem + lane_off + C::TM_DP + 64 * hf + 32 * c, dr);
         tmem_ld_wait();
         reg_fence(dr);
+        if (stamp && c == 0) FA_STAMP(p, T_S_DPLD, t);
         const float4* dlt4 = reinterpret_cast<const float4*>(dlt_t + 32 * c);
 #pragma unroll
         for (int q = 0; q < 32; q += 2) {
@@ -576,10 +594,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                                                p1 * (__uint_as_float(dr[q + 1]) - db));
         }
       }
-      // dS^T over the first 32 of this half's own 64 dP^T columns (A of dK),
-      // and into the shared dS^T tile (A of dQ, read MN-major). At D = 128
-      // this warp's slice of the tile staged a dQ box: its read must be done.
-      tmem_st32(tmem + lane_off + C::TM_DP + 64 * hf, dsk);
+      // dS^T into the shared dS^T tile: the A operand of dQ (read MN-major)
+      // and of dK (read K-major). At D = 128 this warp's slice of the tile
+      // staged a dQ box: its read must be done.
+      if (stamp) FA_STAMP(p, T_S_DSC, t);
       if (C::NBOX > 1) {
         if (lane == 0) bulk_wait_read_all();
         __syncwarp();
@@ -588,8 +606,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int m = 0; m < 8; ++m)
         *reinterpret_cast<uint4*>(ds_row + ((m ^ (r & 7)) << 4)) =
             make_uint4(dsk[4 * m + 0], dsk[4 * m + 1], dsk[4 * m + 2], dsk[4 * m + 3]);
+      if (stamp) FA_STAMP(p, T_S_DSST, t);
       fence_proxy_async_smem();
-      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bars.ds_ready());
       if (stamp) FA_STAMP(p, T_S_DSREADY, t);

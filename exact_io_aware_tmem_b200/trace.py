@@ -24,7 +24,8 @@ import sys
 BWD_KINDS = {
     "P_Q": 0, "P_DO": 1, "M_PREADY": 2, "M_SNEXT": 3, "M_DSREADY": 4, "M_DQ": 5,
     "M_DQFREE": 6, "M_DP": 7, "S_SFULL": 8, "S_PREADY": 9, "S_DQFULL": 10, "S_DQFREE": 11,
-    "S_STAGED": 12, "S_DPFULL": 13, "S_DSREADY": 14, "M_DV": 15,
+    "S_STAGED": 12, "S_DPFULL": 13, "S_DSREADY": 14, "M_DV": 15, "S_SLD": 16, "S_EXPD": 17,
+    "S_DPLD": 18, "S_DSC": 19, "S_DSST": 20,
 }
 FWD_KINDS = {
     "P_K": 0, "P_V": 1, "M_VFULL": 2, "M_PV0": 3, "M_S0": 4, "M_PV1": 5, "M_S1": 6,
@@ -36,11 +37,18 @@ FWD_KINDS = {
 # median of stamp[to][t + dto] - stamp[from][t + dfrom] over the steps t.
 BWD_SPANS = [
     ("dS warps: exponentials of S_t (s_full -> p_ready)", "S_SFULL", 0, "S_PREADY", 0),
+    ("  first 32 scores in registers", "S_SFULL", 0, "S_SLD", 0),
+    ("  -> exponentials of 64 scores done", "S_SLD", 0, "S_EXPD", 0),
+    ("  -> P in TMEM, p_ready", "S_EXPD", 0, "S_PREADY", 0),
     ("dS warps: wait for dQ_{t-1} (p_ready -> dq_full)", "S_PREADY", 0, "S_DQFULL", -1),
     ("dS warps: read dQ_{t-1} out of TMEM", "S_DQFULL", -1, "S_DQFREE", -1),
     ("dS warps: stage dQ_{t-1}, issue reductions", "S_DQFREE", -1, "S_STAGED", -1),
     ("dS warps: wait for dP_t (-> dp_full)", "S_STAGED", -1, "S_DPFULL", 0),
     ("dS warps: dS phase (dp_full -> ds_ready)", "S_DPFULL", 0, "S_DSREADY", 0),
+    ("  first 32 of dP in registers", "S_DPFULL", 0, "S_DPLD", 0),
+    ("  -> dS of 64 formed", "S_DPLD", 0, "S_DSC", 0),
+    ("  -> dS to TMEM issued, staging read done, dS to shared memory", "S_DSC", 0, "S_DSST", 0),
+    ("  -> fences, ds_ready", "S_DSST", 0, "S_DSREADY", 0),
     ("dS warps: wait for S_{t+1} (ds_ready -> s_full)", "S_DSREADY", 0, "S_SFULL", 1),
     ("step period (s_full -> s_full)", "S_SFULL", 0, "S_SFULL", 1),
     ("MMA: p_ready seen after arrival", "S_PREADY", 0, "M_PREADY", 0),
