@@ -292,17 +292,18 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       pb.nxt = page_id(first + 32 + lane);
     };
     // Page id of page pg0 + min(lane, n - 1): the n (<= 8) pages of one tile,
-    // one per lane. pg0 is warp-uniform and never decreases.
+    // one per lane. pg0 is warp-uniform and never decreases. A tile's pages
+    // never straddle two batches (pg0 is a multiple of n, and n divides 32),
+    // so only the current batch is read; the next one is used only when the
+    // batch advances, long after its load was issued.
     auto batch_get = [&](PageBatch& pb, int pg0, int n) -> int {
       while (pg0 >= pb.base + 32) {
         pb.base += 32;
         pb.cur = pb.nxt;
         pb.nxt = page_id(pb.base + 32 + lane);
       }
-      const int off = pg0 + min(lane, n - 1) - pb.base;   // < 32 + 8
-      const int from_cur = __shfl_sync(FULL, pb.cur, off & 31);
-      const int from_nxt = __shfl_sync(FULL, pb.nxt, off & 31);
-      return off < 32 ? from_cur : from_nxt;
+      const int off = pg0 + min(lane, n - 1) - pb.base;   // < 32
+      return __shfl_sync(FULL, pb.cur, off & 31);
     };
     const bool paged = DEC && dec.block_table != nullptr;
     const int box = paged ? min(dec.page, BN) : BN;   // rows per TMA box
