@@ -24,9 +24,9 @@
 //                                                                -> TMEM dK
 // and the fp32 dQ_t partial is added into the caller's fp32 accumulator
 // dQacc [T, H, D] (zeroed by the preprocess kernel; a convert kernel writes
-// dQ = bf16(scale dQacc) afterwards): each dS warp stages its 32 x 32 box of
-// dQ_t in shared memory and one lane adds it with a TMA tensor reduction,
-// which runs on its own while the warp goes on. The accumulation order over
+// dQ = bf16(scale dQacc) afterwards): four dQ warps read it out of TMEM,
+// stage it in 32 x 32 boxes in shared memory, and one lane of each adds its
+// boxes with TMA tensor reductions, which run on their own. The accumulation order over
 // key tiles is not fixed, so dQ is reproducible only to rounding; dK and dV
 // are summed in a fixed order inside one CTA.
 //
@@ -35,12 +35,11 @@
 // before they signal dS_t), and dP_{t+1} waits until they have read dQ_t out.
 // At D = 64 dQ_t has columns of its own.
 //
-// Roles (320 threads):
+// Roles (448 threads):
 //   warps 0-7  dS warps. Thread = key row (TMEM lane) for S^T / dP^T, warps w
 //              and w+4 taking query columns [64 hf, 64 hf + 64). Per step:
-//              exponentials of S^T_t -> P^T_t into TMEM; then the read-out of
-//              dQ_{t-1} (thread = query row), staged for its reduction; then
-//              dS^T_t into the shared dS tile.
+//              exponentials of S^T_t -> P^T_t into TMEM, then dS^T_t into the
+//              shared dS tile.
 //   warp 8     TMA producer: K, V once; Q_t (with the step's LSE and D_i
 //              staged beside it) through a two-stage ring, dO_t through one
 //              stage (dV_t, its last reader, runs long before dP_{t+1}).
@@ -49,6 +48,10 @@
 //              because its read-out gates dP_{t+1}; the exponentials of step
 //              t+1 overlap dQ_t and dK_t, and the dS phase of step t overlaps
 //              dV_t and S_{t+1}.
+//   warps 10-13 dQ warps. Thread = query row of dQ_t (TMEM lane): read-out,
+//              staging and reductions, off the dS warps' path, so that the
+//              exponentials of step t+1 run while dQ_t is read out and dP_{t+1}
+//              is formed.
 #include <limits.h>
 #include <math.h>
 
@@ -62,10 +65,12 @@ namespace {
 namespace fused {
 
 constexpr int BT = 128;        // keys per CTA = query rows per step = TMEM lanes
-constexpr int THREADS = 320;
+constexpr int THREADS = 448;
 constexpr int N_DS = 256;      // dS warps' threads
 constexpr int WARP_TMA = 8;
 constexpr int WARP_MMA = 9;
+constexpr int WARP_DQ0 = 10;   // dQ warps 10-13: TMEM lane quarters 2, 3, 0, 1
+constexpr int N_DQ = 128;      // dQ warps' threads
 constexpr uint32_t TMEM_COLS = 512;
 constexpr unsigned FULL = 0xffffffffu;
 constexpr uint32_t SPAN = BT * 128;   // 128 rows x 128 bytes: one 128-byte swizzle column block
@@ -78,7 +83,7 @@ struct Cfg {
   static constexpr int QS = 2;                       // Q stages (with LSE, D_i)
   static constexpr int GS = 1;                       // dO stages (dO_{t+1} is read after dV_t)
   static constexpr bool ALIAS = D == 128;            // dQ_t formed over dP
-  static constexpr int NBOX = D / 64;                // 32 x 32 fp32 dQ boxes per dS warp per step
+  static constexpr int ROUNDS = D / 64;              // dQ read-out rounds of two 32 x 32 boxes
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr uint32_t TM_DQ = ALIAS ? TM_DP : 256 + 2 * D;
   static constexpr uint32_t OFF_K = 0;
@@ -86,13 +91,13 @@ struct Cfg {
   static constexpr uint32_t OFF_Q = OFF_V + TILE;
   static constexpr uint32_t OFF_DO = OFF_Q + QS * TILE;
   static constexpr uint32_t OFF_DS = OFF_DO + GS * TILE;       // dS^T: 128 keys x 128 queries bf16
-  static constexpr uint32_t OFF_STG = OFF_DS + 2 * SPAN;       // dQ staging: 4 KB per dS warp
+  static constexpr uint32_t OFF_STG = OFF_DS + 2 * SPAN;       // dQ staging: 8 KB per dQ warp
   static constexpr uint32_t OFF_LSE = OFF_STG + 8 * 4096;      // float [QS][BT]: LSE * log2(e)
   static constexpr uint32_t OFF_DLT = OFF_LSE + QS * BT * 4;   // float [QS][BT]: D_i
   static constexpr uint32_t OFF_BAR = OFF_DLT + QS * BT * 4;
   // kv_full, q_full[QS], q_empty[QS], do_full[GS], do_empty[GS], s_full,
-  // dp_full, p_ready, ds_ready, dq_full, dq_free, dkv_done, ds_free
-  static constexpr int NBAR = 1 + 2 * QS + 2 * GS + 8;
+  // dp_full, p_ready, ds_ready, dq_full, dq_free, dkv_done
+  static constexpr int NBAR = 1 + 2 * QS + 2 * GS + 7;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
   // No alignment slack: the dynamic shared memory must start on a 1024-byte
   // boundary (128-byte swizzle atoms); the kernel checks and reports.
@@ -117,15 +122,14 @@ struct Bars {
   __device__ uint32_t dq_full() const { return b + 8u * (5 + 2 * C::QS + 2 * C::GS); }
   __device__ uint32_t dq_free() const { return b + 8u * (6 + 2 * C::QS + 2 * C::GS); }
   __device__ uint32_t dkv_done() const { return b + 8u * (7 + 2 * C::QS + 2 * C::GS); }
-  // dK_t has read the shared dS^T tile (which then takes a staged dQ box).
-  __device__ uint32_t ds_free() const { return b + 8u * (8 + 2 * C::QS + 2 * C::GS); }
 };
 
-// Event kinds of the debug build's stamps (one per step t unless noted).
+// Event kinds of the debug build's stamps (one per step t unless noted):
+// P_ producer, M_ MMA warp, S_ dS warps, Q_ dQ warps.
 enum : int {
   T_P_Q = 0, T_P_DO = 1, T_M_PREADY = 2, T_M_SNEXT = 3 /* S_{t+1}, index t+1 */,
   T_M_DSREADY = 4, T_M_DQ = 5, T_M_DQFREE = 6, T_M_DP = 7 /* dP_{t+1}, index t+1 */,
-  T_S_SFULL = 8, T_S_PREADY = 9, T_S_DQFULL = 10, T_S_DQFREE = 11, T_S_STAGED = 12,
+  T_S_SFULL = 8, T_S_PREADY = 9, T_Q_DQFULL = 10, T_Q_DQFREE = 11, T_Q_STAGED = 12,
   T_S_DPFULL = 13, T_S_DSREADY = 14, T_M_DV = 15, T_S_SLD = 16 /* scores in registers */,
   T_S_EXPD = 17 /* exponentials done */, T_S_DPLD = 18 /* dP in registers */,
   T_S_DSC = 19 /* dS formed */, T_S_DSST = 20 /* dS stored to shared memory */
@@ -134,8 +138,7 @@ enum : int {
 enum : unsigned {
   W_KV = 0x40100, W_QEMPTY = 0x40200, W_QFULL = 0x40300, W_SFULL = 0x40400, W_PREADY = 0x40500,
   W_DPFULL = 0x40600, W_DSREADY = 0x40700, W_DKV = 0x40800, W_DOFULL = 0x40900,
-  W_DOEMPTY = 0x40A00, W_DQFULL = 0x40B00, W_DQFREE = 0x40C00, BAD_ALIGN = 0x40D00,
-  W_DSFREE = 0x40E00
+  W_DOEMPTY = 0x40A00, W_DQFULL = 0x40B00, W_DQFREE = 0x40C00, BAD_ALIGN = 0x40D00
 };
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DevErr& e,
@@ -203,8 +206,11 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// 14 warps put four on each of two SM sub-partitions, whose 16K registers
+// then allow 128 per thread: the bound of 512 threads holds the compiler to
+// that.
 template <int D>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -259,9 +265,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bars.p_ready(), N_DS);
     mbar_init(bars.ds_ready(), N_DS);
     mbar_init(bars.dq_full(), 1);
-    mbar_init(bars.dq_free(), N_DS);
+    mbar_init(bars.dq_free(), N_DQ);
     mbar_init(bars.dkv_done(), 1);
-    mbar_init(bars.ds_free(), 1);
     fence_mbar_init();
   }
   if (warp == WARP_MMA) {
@@ -433,7 +438,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                   sdesc_add(q_mn, st * C::TILE + kk * 2048), ID_KV, (t > 0 || kk > 0) ? 1u : 0u);
       }
       tc_commit_if(leader, bars.q_empty(st));
-      tc_commit_if(leader, bars.ds_free());
       if (more) {
         if (C::ALIAS) {
           // dP_{t+1} overwrites dQ_t: wait until it has been read out.
@@ -449,12 +453,67 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
     tc_commit_if(leader, bars.dkv_done());
+  } else if (warp >= WARP_DQ0) {
+    // ------------------------------------------------------------ dQ warps ---
+    // Thread = query row (warp & 3) * 32 + lane of the step's tile. Each
+    // round reads two 32 x 32 boxes of dQ_t (fp32) out of TMEM, stages them
+    // 128-byte swizzled in this warp's 8 KB of the staging area, and one lane
+    // adds them into dQacc with TMA tensor reductions, which run on their own.
+    // dq_free goes out as soon as the last round is in registers.
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t stg = sbase + C::OFF_STG + (warp - WARP_DQ0) * 8192u;
+    const bool stamp = warp == WARP_DQ0 && lane == 0;   // debug stamps
+    for (int t = 0; t < n_steps; ++t) {
+      if (!warp_wait(bars.dq_full(), t & 1, p.err, abort, W_DQFULL)) break;
+      if (stamp) FA_STAMP(p, T_Q_DQFULL, t);
+      tc_fence_after();
+      const int h = hk * g + t / n_qt;
+      const int row0 = sq.start + (i0 + t % n_qt) * BT + (warp & 3) * 32;
+      // Rows past the sequence's end hold exact zeros (their dS rows are
+      // zero), so adding them to the next sequence's rows changes nothing;
+      // rows past the tensor are clipped by the copy. A box wholly past the
+      // sequence is not added at all.
+      const bool add = row0 < sq.start + sq.len;
+#pragma unroll
+      for (int rd = 0; rd < C::ROUNDS; ++rd) {
+        uint32_t a[2][32];
+        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * rd, a[0]);
+        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * rd + 32, a[1]);
+        tmem_ld_wait();
+        reg_fence(a[0]);
+        reg_fence(a[1]);
+        if (rd == C::ROUNDS - 1) {
+          tc_fence_before();
+          mbar_arrive(bars.dq_free());
+          if (stamp) FA_STAMP(p, T_Q_DQFREE, t);
+        }
+        // The slots' previous boxes must have been read.
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            st_shared_v4(stg + c * 4096u + lane * 128 + ((m ^ (lane & 7)) << 4), a[c][4 * m],
+                         a[c][4 * m + 1], a[c][4 * m + 2], a[c][4 * m + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && add &&
+            FA_CHECK(p, row0 >= 0 && row0 < p.total && h < p.H, 0xDB0402u)) {
+          tma_reduce_add_2d(&tm_dqa, stg, h * D + 64 * rd, row0);
+          tma_reduce_add_2d(&tm_dqa, stg + 4096u, h * D + 64 * rd + 32, row0);
+        }
+        if (lane == 0) bulk_commit();
+      }
+      if (stamp) FA_STAMP(p, T_Q_STAGED, t);
+    }
+    // The reductions read this CTA's shared memory: all must be done before exit.
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ dS warps ---
     // Key-side work: thread = key row r (TMEM lane); warps w and w+4 take the
-    // query columns [64 hf, 64 hf + 64) of the step. Read-out of dQ_t: thread
-    // = query row (warp & 3) * 32 + lane of the step's tile, columns
-    // [hf D / 2, hf D / 2 + D / 2) of the head dim.
+    // query columns [64 hf, 64 hf + 64) of the step.
     const int r = threadIdx.x & (BT - 1);
     const int hf = threadIdx.x >> 7;
     const int kpos = j * BT + r;
@@ -470,58 +529,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // queries per 128-byte block, 16-byte chunks XOR-swizzled by row & 7).
     uint8_t* ds_row = smem + C::OFF_DS + hf * SPAN + r * 128;
 
-    // Adds the dQ partial of step tq (in TMEM) into dQacc. Thread = query row
-    // (warp & 3) * 32 + lane of the step's tile; the warp's 32 rows x 32
-    // columns form one box, staged 128-byte swizzled in shared memory and
-    // added by a TMA tensor reduction, which runs on its own while the warp
-    // goes on. At D = 128 the second box of a step is staged in this warp's
-    // 4 KB slice of the dS tile (free until dS of the next step, and written
-    // then only by this warp), the first in its slice of the staging area.
-    const uint32_t stg[2] = {sbase + C::OFF_STG + warp * 4096u, sbase + C::OFF_DS + warp * 4096u};
     const bool stamp = threadIdx.x == 0;   // debug stamps: lane 0 of warp 0
-    auto drain_dq = [&](int tq) -> bool {
-      if (!warp_wait(bars.dq_full(), tq & 1, p.err, abort, W_DQFULL)) return false;
-      if (stamp) FA_STAMP(p, T_S_DQFULL, tq);
-      tc_fence_after();
-      uint32_t a[C::NBOX][32];
-#pragma unroll
-      for (int c = 0; c < C::NBOX; ++c)
-        tmem_ld32(tmem + lane_off + C::TM_DQ + hf * (D / 2) + 32 * c, a[c]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int c = 0; c < C::NBOX; ++c) reg_fence(a[c]);
-      tc_fence_before();
-      mbar_arrive(bars.dq_free());
-      if (stamp) FA_STAMP(p, T_S_DQFREE, tq);
-      const int h = hk * g + tq / n_qt;
-      const int row0 = sq.start + (i0 + tq % n_qt) * BT + (warp & 3) * 32;
-      // The staging slices' previous contents (a step back) must have been read.
-      if (lane == 0) bulk_wait_read_all();
-      __syncwarp();
-      // The second box goes into this warp's slice of the dS^T tile: dK_tq
-      // must have finished reading it.
-      if (C::NBOX > 1 && !warp_wait(bars.ds_free(), tq & 1, p.err, abort, W_DSFREE)) return false;
-#pragma unroll
-      for (int c = 0; c < C::NBOX; ++c) {
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-          st_shared_v4(stg[c] + lane * 128 + ((m ^ (lane & 7)) << 4), a[c][4 * m], a[c][4 * m + 1],
-                       a[c][4 * m + 2], a[c][4 * m + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        // Rows past the sequence's end hold exact zeros (their dS rows are
-        // zero), so adding them to the next sequence's rows changes nothing;
-        // rows past the tensor are clipped by the copy. A box wholly past the
-        // sequence is not added at all.
-        if (lane == 0 && row0 < sq.start + sq.len &&
-            FA_CHECK(p, row0 >= 0 && row0 < p.total && h < p.H, 0xDB0402u))
-          tma_reduce_add_2d(&tm_dqa, stg[c], h * D + hf * (D / 2) + 32 * c, row0);
-      }
-      if (lane == 0) bulk_commit();
-      if (stamp) FA_STAMP(p, T_S_STAGED, tq);
-      return true;
-    };
-
     bool ok = true;
     for (int t = 0; t < n_steps && ok; ++t) {
       const int st = t % C::QS;
@@ -566,8 +574,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(bars.p_ready());
       if (stamp) FA_STAMP(p, T_S_PREADY, t);
 
-      // dQ of the previous step: its product ran under this step's exponentials.
-      if (t > 0 && !(ok = drain_dq(t - 1))) break;
 
       if (!(ok = warp_wait(bars.dp_full(), t & 1, p.err, abort, W_DPFULL))) break;
       if (stamp) FA_STAMP(p, T_S_DPFULL, t);
@@ -595,13 +601,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // dS^T into the shared dS^T tile: the A operand of dQ (read MN-major)
-      // and of dK (read K-major). At D = 128 this warp's slice of the tile
-      // staged a dQ box: its read must be done.
+      // and of dK (read K-major). dP_t completing means dQ_{t-1} and dK_{t-1}
+      // (issued before it) have read the tile.
       if (stamp) FA_STAMP(p, T_S_DSC, t);
-      if (C::NBOX > 1) {
-        if (lane == 0) bulk_wait_read_all();
-        __syncwarp();
-      }
 #pragma unroll
       for (int m = 0; m < 8; ++m)
         *reinterpret_cast<uint4*>(ds_row + ((m ^ (r & 7)) << 4)) =
@@ -612,10 +614,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(bars.ds_ready());
       if (stamp) FA_STAMP(p, T_S_DSREADY, t);
     }
-    if (ok && n_steps > 0) ok = drain_dq(n_steps - 1);
-    // The reductions read this CTA's shared memory: all must be done before exit.
-    if (lane == 0) bulk_wait_all();
-    __syncwarp();
     // --------------------------------------------------- dK / dV epilogue ---
     if (ok && warp_wait(bars.dkv_done(), 0, p.err, abort, W_DKV)) {
       tc_fence_after();

@@ -23,8 +23,8 @@ import sys
 # Event kinds, as numbered in the kernels' sources.
 BWD_KINDS = {
     "P_Q": 0, "P_DO": 1, "M_PREADY": 2, "M_SNEXT": 3, "M_DSREADY": 4, "M_DQ": 5,
-    "M_DQFREE": 6, "M_DP": 7, "S_SFULL": 8, "S_PREADY": 9, "S_DQFULL": 10, "S_DQFREE": 11,
-    "S_STAGED": 12, "S_DPFULL": 13, "S_DSREADY": 14, "M_DV": 15, "S_SLD": 16, "S_EXPD": 17,
+    "M_DQFREE": 6, "M_DP": 7, "S_SFULL": 8, "S_PREADY": 9, "Q_DQFULL": 10, "Q_DQFREE": 11,
+    "Q_STAGED": 12, "S_DPFULL": 13, "S_DSREADY": 14, "M_DV": 15, "S_SLD": 16, "S_EXPD": 17,
     "S_DPLD": 18, "S_DSC": 19, "S_DSST": 20,
 }
 FWD_KINDS = {
@@ -40,26 +40,25 @@ BWD_SPANS = [
     ("  first 32 scores in registers", "S_SFULL", 0, "S_SLD", 0),
     ("  -> exponentials of 64 scores done", "S_SLD", 0, "S_EXPD", 0),
     ("  -> P in TMEM, p_ready", "S_EXPD", 0, "S_PREADY", 0),
-    ("dS warps: wait for dQ_{t-1} (p_ready -> dq_full)", "S_PREADY", 0, "S_DQFULL", -1),
-    ("dS warps: read dQ_{t-1} out of TMEM", "S_DQFULL", -1, "S_DQFREE", -1),
-    ("dS warps: stage dQ_{t-1}, issue reductions", "S_DQFREE", -1, "S_STAGED", -1),
-    ("dS warps: wait for dP_t (-> dp_full)", "S_STAGED", -1, "S_DPFULL", 0),
+    ("dS warps: wait for dP_t (p_ready -> dp_full)", "S_PREADY", 0, "S_DPFULL", 0),
     ("dS warps: dS phase (dp_full -> ds_ready)", "S_DPFULL", 0, "S_DSREADY", 0),
     ("  first 32 of dP in registers", "S_DPFULL", 0, "S_DPLD", 0),
     ("  -> dS of 64 formed", "S_DPLD", 0, "S_DSC", 0),
-    ("  -> dS to TMEM issued, staging read done, dS to shared memory", "S_DSC", 0, "S_DSST", 0),
+    ("  -> dS to shared memory", "S_DSC", 0, "S_DSST", 0),
     ("  -> fences, ds_ready", "S_DSST", 0, "S_DSREADY", 0),
     ("dS warps: wait for S_{t+1} (ds_ready -> s_full)", "S_DSREADY", 0, "S_SFULL", 1),
     ("step period (s_full -> s_full)", "S_SFULL", 0, "S_SFULL", 1),
+    ("dQ warps: read-out of dQ_t (dq_full -> dq_free)", "Q_DQFULL", 0, "Q_DQFREE", 0),
+    ("dQ warps: staged, reductions issued (dq_free -> staged)", "Q_DQFREE", 0, "Q_STAGED", 0),
     ("MMA: p_ready seen after arrival", "S_PREADY", 0, "M_PREADY", 0),
     ("MMA: dV_t issued (p_ready seen -> issued)", "M_PREADY", 0, "M_DV", 0),
     ("MMA: S_{t+1} issued after dV_t", "M_DV", 0, "M_SNEXT", 1),
     ("MMA: ds_ready seen after arrival", "S_DSREADY", 0, "M_DSREADY", 0),
-    ("MMA: dK_t, dQ_t issued (ds_ready seen -> dQ issued)", "M_DSREADY", 0, "M_DQ", 0),
-    ("MMA: dq_free seen after arrival", "S_DQFREE", 0, "M_DQFREE", 0),
+    ("MMA: dQ_t issued (ds_ready seen -> dQ issued)", "M_DSREADY", 0, "M_DQ", 0),
+    ("MMA: dq_free seen after arrival", "Q_DQFREE", 0, "M_DQFREE", 0),
     ("MMA: dP_{t+1} issued after dq_free", "M_DQFREE", 0, "M_DP", 1),
     ("tensor: S_{t+1} issue -> s_full seen", "M_SNEXT", 1, "S_SFULL", 1),
-    ("tensor: dQ_t issue -> dq_full seen", "M_DQ", 0, "S_DQFULL", 0),
+    ("tensor: dQ_t issue -> dq_full seen", "M_DQ", 0, "Q_DQFULL", 0),
     ("tensor: dP_{t+1} issue -> dp_full seen", "M_DP", 1, "S_DPFULL", 1),
     ("producer: Q_{t+1} issued before S_{t+1} issue", "P_Q", 1, "M_SNEXT", 1),
     ("producer: dO_{t+1} issued before dP_{t+1} issue", "P_DO", 1, "M_DP", 1),
