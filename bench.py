@@ -681,6 +681,7 @@ def run_fp8(args, name, w) -> None:
     # by the length of the timed region).
     bf16_peak, peak_kind = tensor_peak(peaks, max_ms / 1e3)
     peak = bf16_peak / 0.75
+    p1_bytes = sum(3 * t.numel() + 4 * s_.numel() for t, s_ in ((q, qs), (k, ks)))
     achieved = fwd_fl / (f_ms / 1e3) / 1e12
     line = {
         "metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -700,6 +701,12 @@ def run_fp8(args, name, w) -> None:
                      "peak_kind": f"{peaks['source']} {peak_kind} bf16 / 0.75 (E4M3 Q K^T at the "
                                   f"nominal 2x rate, bf16 P V)",
                      "traffic": recorded_traffic("fp8_fwd", name)},
+        # Pass 1 is HBM-bound: it reads bf16 Q and K once and writes their
+        # E4M3 codes and steps.
+        "pass1_roofline": {"kernel": "fp8_quantize_kernel (Q and K)", "bound": "hbm",
+                           "achieved": p1_bytes / (q_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": p1_bytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                           "algorithmic_bytes": p1_bytes},
         "cpu_baseline": cpu,
         "e2e": {"value": fwd_fl * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

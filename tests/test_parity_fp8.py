@@ -46,6 +46,44 @@ def test_quantize_codes_and_steps_are_exact(B, N, Hx, D):
     np.testing.assert_array_equal(_codes_as_values(x8), xh)
 
 
+def _hard_blocks(seed: int, n_blocks: int, D: int) -> torch.Tensor:
+    """n_blocks blocks of 128 tokens x D (one head), each with its own max |x|
+    and elements drawn uniformly over bf16 bit patterns below it (every
+    exponent down to the subnormals), so x / Delta lands everywhere on the
+    E4M3 grid, at its rounding midpoints and in its subnormal range. Block 0
+    holds the midpoints of the grid and their bf16 neighbours with Delta = 1
+    (max |x| = 448); block 1 has a max |x| whose Delta is an fp32 subnormal."""
+    g = torch.Generator().manual_seed(seed)
+    per = 128 * D
+    amax_bits = torch.randint(0x3000, 0x4700, (n_blocks,), generator=g, dtype=torch.int32)
+    amax_bits[1] = 0x0100                                      # 2^-125: Delta an fp32 subnormal
+    amax = (amax_bits << 16).view(torch.float32)
+    bits = torch.randint(0, 1 << 30, (n_blocks, per), generator=g, dtype=torch.int32)
+    bits = bits % (amax_bits[:, None] + 1)                     # bf16 patterns in [0, max |x|]
+    x = (bits << 16).view(torch.float32)
+    # grid midpoints of E4M3 (normal and subnormal) and their bf16 neighbours
+    grid = torch.arange(0, 127, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    grid = grid.to(torch.float32)
+    mid = (grid[:-1] + grid[1:]) / 2
+    nb = torch.cat([mid, torch.nextafter(mid.bfloat16().float(), torch.tensor(0.0)),
+                    torch.nextafter(mid.bfloat16().float(), torch.tensor(1e9))]).bfloat16().float()
+    x[0, : nb.numel()] = nb
+    amax[0] = 448.0
+    x[:, -1] = amax                                            # the block's max
+    sign = torch.randint(0, 2, x.shape, generator=g).float() * 2 - 1
+    return (x * sign).bfloat16()
+
+
+def test_quantize_codes_exact_on_every_exponent_and_midpoint():
+    D, n_blocks = 128, 24
+    x = _hard_blocks(5, n_blocks, D).view(n_blocks * 128, 1, D)
+    x8, sc = fa.fp8_quantize(x.cuda(), 1, n_blocks * 128)
+    torch.cuda.synchronize()
+    xh, d = of.quantize_blocks(x, 1, n_blocks * 128)
+    np.testing.assert_array_equal(sc.cpu().numpy(), d)
+    np.testing.assert_array_equal(_codes_as_values(x8), xh)
+
+
 def _fp8_case(inp, B, N, causal, scale):
     q8, qs = fa.fp8_quantize(inp.q.cuda(), B, N)
     k8, ks = fa.fp8_quantize(inp.k.cuda(), B, N)
