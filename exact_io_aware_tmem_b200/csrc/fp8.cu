@@ -35,26 +35,44 @@ constexpr int QTHREADS = 256;
 // rounding midpoint of the E4M3 grid within the bracket, about one element in
 // 10^5) the caller divides. Returns the four codes of the low end; *same is
 // whether the high end agrees.
+// Four floats -> four E4M3 codes (round to nearest even, saturating), a in
+// byte 0.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
+      "mov.b32 %0, {l, h};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t codes4(uint32_t w0, uint32_t w1, float r_lo, float r_hi,
                                            bool* same) {
   const float x0 = __uint_as_float(w0 << 16), x1 = __uint_as_float(w0 & 0xffff0000u);
   const float x2 = __uint_as_float(w1 << 16), x3 = __uint_as_float(w1 & 0xffff0000u);
-  const uint32_t lo = pack_e4m3x2(__fmul_rn(x0, r_lo), __fmul_rn(x1, r_lo)) |
-                      (static_cast<uint32_t>(pack_e4m3x2(__fmul_rn(x2, r_lo), __fmul_rn(x3, r_lo)))
-                       << 16);
-  const uint32_t hi = pack_e4m3x2(__fmul_rn(x0, r_hi), __fmul_rn(x1, r_hi)) |
-                      (static_cast<uint32_t>(pack_e4m3x2(__fmul_rn(x2, r_hi), __fmul_rn(x3, r_hi)))
-                       << 16);
+  const uint32_t lo = pack_e4m3x4(__fmul_rn(x0, r_lo), __fmul_rn(x1, r_lo), __fmul_rn(x2, r_lo),
+                                  __fmul_rn(x3, r_lo));
+  const uint32_t hi = pack_e4m3x4(__fmul_rn(x0, r_hi), __fmul_rn(x1, r_hi), __fmul_rn(x2, r_hi),
+                                  __fmul_rn(x3, r_hi));
   *same = lo == hi;
   return lo;
+}
+
+// Elementwise max of two bf16 pairs.
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 // The same four codes by IEEE division.
 __device__ __forceinline__ uint32_t codes4_div(uint32_t w0, uint32_t w1, float delta) {
   const float x0 = __uint_as_float(w0 << 16), x1 = __uint_as_float(w0 & 0xffff0000u);
   const float x2 = __uint_as_float(w1 << 16), x3 = __uint_as_float(w1 & 0xffff0000u);
-  return pack_e4m3x2(__fdiv_rn(x0, delta), __fdiv_rn(x1, delta)) |
-         (static_cast<uint32_t>(pack_e4m3x2(__fdiv_rn(x2, delta), __fdiv_rn(x3, delta))) << 16);
+  return pack_e4m3x4(__fdiv_rn(x0, delta), __fdiv_rn(x1, delta), __fdiv_rn(x2, delta),
+                     __fdiv_rn(x3, delta));
 }
 
 // One CTA per (sequence, 128-token block, head). The block (at most
@@ -63,7 +81,7 @@ __device__ __forceinline__ uint32_t codes4_div(uint32_t w0, uint32_t w1, float d
 // PER_ROW: D / 8 when fixed at compile time (the addresses then take shifts),
 // 0 for any D (a division per address).
 template <int VPT, int PER_ROW>
-__global__ void __launch_bounds__(QTHREADS, 32 / VPT)
+__global__ void __launch_bounds__(QTHREADS, VPT >= 8 ? 32 / VPT : 6)
     fp8_quantize_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ x8,
                         float* __restrict__ scale, int N, int Hx, int D, int nb) {
   static_assert(VPT <= 16, "one bit per four elements");
@@ -78,26 +96,37 @@ __global__ void __launch_bounds__(QTHREADS, 32 / VPT)
   const int rows = min(QBLOCK, N - r0);
   const int per_row = PER_ROW ? PER_ROW : D / 8;
   const int n = rows * per_row;
-  auto offset = [&](int i) -> size_t {   // element offset of the i-th group of 8
-    const int row = i / per_row;
-    return (static_cast<size_t>(b) * N + r0 + row) * Hx * D + static_cast<size_t>(h) * D +
-           (i % per_row) * 8;
+  // Element offset of this thread's k-th group of 8 (group i = threadIdx.x +
+  // k QTHREADS of the block). With a compile-time row width that divides
+  // QTHREADS, step k moves the thread down QTHREADS / PER_ROW whole rows: a
+  // fixed stride.
+  const size_t base = (static_cast<size_t>(b) * N + r0) * Hx * D + static_cast<size_t>(h) * D;
+  const size_t row_pitch = static_cast<size_t>(Hx) * D;
+  auto offset = [&](int k) -> size_t {
+    if constexpr (PER_ROW != 0 && QTHREADS % (PER_ROW ? PER_ROW : 1) == 0) {
+      return base + (threadIdx.x / PER_ROW + static_cast<size_t>(k) * (QTHREADS / PER_ROW)) *
+                        row_pitch +
+             (threadIdx.x % PER_ROW) * 8;
+    } else {
+      const int i = threadIdx.x + k * QTHREADS;
+      return base + static_cast<size_t>(i / per_row) * row_pitch + (i % per_row) * 8;
+    }
   };
   uint4 v[VPT];
 #pragma unroll
   for (int k = 0; k < VPT; ++k) {
     const int i = threadIdx.x + k * QTHREADS;
-    v[k] = i < n ? __ldcs(reinterpret_cast<const uint4*>(x + offset(i))) : make_uint4(0, 0, 0, 0);
+    v[k] = i < n ? __ldcs(reinterpret_cast<const uint4*>(x + offset(k))) : make_uint4(0, 0, 0, 0);
   }
-  // max |x| over bf16 bit patterns: with the sign bits cleared, two halves
-  // at a time, the patterns order as the values do.
+  // max |x|: bf16 pairs with their sign bits cleared, two at a time; then
+  // the bit patterns of the two non-negative halves order as their values.
   uint32_t m2 = 0;
 #pragma unroll
   for (int k = 0; k < VPT; ++k) {
-    m2 = __vmaxu2(m2, v[k].x & 0x7fff7fffu);
-    m2 = __vmaxu2(m2, v[k].y & 0x7fff7fffu);
-    m2 = __vmaxu2(m2, v[k].z & 0x7fff7fffu);
-    m2 = __vmaxu2(m2, v[k].w & 0x7fff7fffu);
+    m2 = max_bf16x2(m2, v[k].x & 0x7fff7fffu);
+    m2 = max_bf16x2(m2, v[k].y & 0x7fff7fffu);
+    m2 = max_bf16x2(m2, v[k].z & 0x7fff7fffu);
+    m2 = max_bf16x2(m2, v[k].w & 0x7fff7fffu);
   }
   uint32_t amax_bits = max(m2 << 16, m2 & 0xffff0000u);
   __shared__ uint32_t red[QTHREADS / 32];
@@ -127,7 +156,7 @@ __global__ void __launch_bounds__(QTHREADS, 32 / VPT)
       const uint32_t c0 = codes4(v[k].x, v[k].y, r_lo, r_hi, &s0);
       const uint32_t c1 = codes4(v[k].z, v[k].w, r_lo, r_hi, &s1);
       redo |= (s0 && normal ? 0u : 1u << (2 * k)) | (s1 && normal ? 0u : 2u << (2 * k));
-      *reinterpret_cast<uint2*>(x8 + offset(i)) = make_uint2(c0, c1);
+      *reinterpret_cast<uint2*>(x8 + offset(k)) = make_uint2(c0, c1);
     }
   }
   // The four-element groups whose bracket holds a rounding midpoint (exact
@@ -140,7 +169,7 @@ __global__ void __launch_bounds__(QTHREADS, 32 / VPT)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         if (redo & (1u << (2 * k + e))) {
-          const size_t o = offset(threadIdx.x + k * QTHREADS) + 4 * e;
+          const size_t o = offset(k) + 4 * e;
           *reinterpret_cast<uint32_t*>(x8 + o) =
               codes4_div(e ? v[k].z : v[k].x, e ? v[k].w : v[k].y, delta);
         }

@@ -32,8 +32,9 @@ def _codes_as_values(x8: torch.Tensor) -> np.ndarray:
     return x8.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
 
 
+# The last two cases are a few thousand blocks (several waves of CTAs).
 @pytest.mark.parametrize("B,N,Hx,D", [(2, 300, 3, 128), (1, 128, 2, 64), (3, 1, 1, 128),
-                                      (1, 1000, 4, 8)])
+                                      (1, 1000, 4, 8), (1, 4096, 64, 128), (2, 2000, 64, 64)])
 def test_quantize_codes_and_steps_are_exact(B, N, Hx, D):
     inp = random_case(7 + N, dtype="bf16", lengths=[N] * B, H=Hx, H_kv=Hx, D=D, varlen=False,
                       std=3.0)
@@ -52,11 +53,13 @@ def _hard_blocks(seed: int, n_blocks: int, D: int) -> torch.Tensor:
     exponent down to the subnormals), so x / Delta lands everywhere on the
     E4M3 grid, at its rounding midpoints and in its subnormal range. Block 0
     holds the midpoints of the grid and their bf16 neighbours with Delta = 1
-    (max |x| = 448); block 1 has a max |x| whose Delta is an fp32 subnormal."""
+    (max |x| = 448); block 1 has a max |x| whose Delta is an fp32 subnormal,
+    block 2 a max |x| that is itself a bf16 subnormal."""
     g = torch.Generator().manual_seed(seed)
     per = 128 * D
     amax_bits = torch.randint(0x3000, 0x4700, (n_blocks,), generator=g, dtype=torch.int32)
     amax_bits[1] = 0x0100                                      # 2^-125: Delta an fp32 subnormal
+    amax_bits[2] = 0x0045                                      # a bf16 subnormal max |x|
     amax = (amax_bits << 16).view(torch.float32)
     bits = torch.randint(0, 1 << 30, (n_blocks, per), generator=g, dtype=torch.int32)
     bits = bits % (amax_bits[:, None] + 1)                     # bf16 patterns in [0, max |x|]
