@@ -128,20 +128,25 @@ KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "decode": ("fwd_bf16.cu", "common.cuh", "params.h"),
-                  "fp8_fwd": ("fwd_bf16.cu", "common.cuh", "params.h")}
+                  "fp8_fwd": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "fp8_quantize_kernel": ("fp8.cu", "common.cuh", "params.h")}
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged."""
+    """DRAM bytes per launch from a committed ncu capture of this kernel on this
+    workload (one record, or a list of records, per kernel), if the kernel is
+    unchanged since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f)[kernel]
+            recs = json.load(f)[kernel]
     except (OSError, KeyError, ValueError):
         return None
-    if rec.get("workload") != workload or rec.get("source_sha") != source_sha(*KERNEL_SOURCES[kernel]):
-        return None
-    return rec.get("bytes_per_launch")
+    for rec in recs if isinstance(recs, list) else [recs]:
+        if rec.get("workload") == workload and \
+                rec.get("source_sha") == source_sha(*KERNEL_SOURCES[kernel]):
+            return rec.get("bytes_per_launch")
+    return None
 
 
 class ClockSampler:
@@ -706,7 +711,10 @@ def run_fp8(args, name, w) -> None:
         "pass1_roofline": {"kernel": "fp8_quantize_kernel (Q and K)", "bound": "hbm",
                            "achieved": p1_bytes / (q_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": p1_bytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                           "algorithmic_bytes": p1_bytes},
+                           "algorithmic_bytes": p1_bytes,
+                           # one launch quantises one of the two tensors
+                           "traffic": (lambda t: None if t is None else 2 * t)(
+                               recorded_traffic("fp8_quantize_kernel", name))},
         "cpu_baseline": cpu,
         "e2e": {"value": fwd_fl * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "steps": e2e_steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

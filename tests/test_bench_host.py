@@ -101,6 +101,12 @@ def test_recorded_traffic_needs_matching_source(monkeypatch, tmp_path):
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     assert bench.recorded_traffic("bwd_dkdv_kernel", "w") == 5
     assert bench.recorded_traffic("bwd_dkdv_kernel", "other") is None
+    # several workloads of one kernel: a list of records
+    rec["bwd_dkdv_kernel"] = [dict(rec["bwd_dkdv_kernel"]),
+                              {"workload": "v", "source_sha": "fresh", "bytes_per_launch": 7}]
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("bwd_dkdv_kernel", "w") == 5
+    assert bench.recorded_traffic("bwd_dkdv_kernel", "v") == 7
     assert real_root
 
 
