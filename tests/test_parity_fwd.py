@@ -109,11 +109,13 @@ def test_bf16_varlen_ragged(D, causal):
     check_full(inp, causal, D ** -0.5, len(lengths), 0, O_TOL_BF16, LSE_TOL_BF16)
 
 
-def test_bf16_large_logits_rescale():
-    # Logit std ~ 8: the running max moves often and the O rescale path runs.
-    inp = random_case(3, dtype="bf16", lengths=[640], H=2, H_kv=2, D=128, varlen=False, std=2.8)
+@pytest.mark.parametrize("D", [64, 128])
+def test_bf16_large_logits_rescale(D):
+    # Logit std ~ 8: the running max moves often and the O rescale path runs
+    # (at D = 64 in each softmax group's own accumulator).
+    inp = random_case(3, dtype="bf16", lengths=[640], H=2, H_kv=2, D=D, varlen=False, std=2.8)
     for causal in (False, True):
-        check_full(inp, causal, 128 ** -0.5, 1, 640, O_TOL_BF16, LSE_TOL_BF16)
+        check_full(inp, causal, D ** -0.5, 1, 640, O_TOL_BF16, LSE_TOL_BF16)
 
 
 def test_bf16_custom_scale():
