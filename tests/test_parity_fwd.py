@@ -110,6 +110,17 @@ def test_bf16_varlen_ragged(D, causal):
 
 
 @pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bf16_many_pairs_ragged(D, causal):
+    # More query-tile pairs than SMs, so a persistent CTA works on several
+    # pairs in turn, many of them with an empty second tile.
+    lengths = [int(x) for x in np.random.default_rng(12).integers(1, 700, size=48)]
+    lengths[3] = 0
+    inp = random_case(13, dtype="bf16", lengths=lengths, H=8, H_kv=4, D=D, varlen=True)
+    check_full(inp, causal, D ** -0.5, len(lengths), 0, O_TOL_BF16, LSE_TOL_BF16)
+
+
+@pytest.mark.parametrize("D", [64, 128])
 def test_bf16_large_logits_rescale(D):
     # Logit std ~ 8: the running max moves often and the O rescale path runs
     # (at D = 64 in each softmax group's own accumulator).
