@@ -24,34 +24,39 @@
 //                                                                -> TMEM dK
 // and the fp32 dQ_t partial is added into the caller's fp32 accumulator
 // dQacc [T, H, D] (zeroed by the preprocess kernel; a convert kernel writes
-// dQ = bf16(scale dQacc) afterwards): four dQ warps read it out of TMEM,
-// stage it in 32 x 32 boxes in shared memory, and one lane of each adds its
-// boxes with TMA tensor reductions, which run on their own. The accumulation order over
+// dQ = bf16(scale dQacc) afterwards): four dQ warps read it out of TMEM in
+// one go, stage it in 32 x 32 boxes in shared memory, and one lane of each
+// adds its boxes with TMA tensor reductions, which run on their own. The accumulation order over
 // key tiles is not fixed, so dQ is reproducible only to rounding; dK and dV
 // are summed in a fixed order inside one CTA.
 //
 // TMEM columns: S [0,128), dP [128,256), dV, dK after them. At D = 128 the
 // 512 columns are full, so dQ_t is formed over dP (the dS warps have read dP_t
-// before they signal dS_t), and dP_{t+1} waits until they have read dQ_t out.
+// before they signal dS_t), and dP_{t+1} waits until dQ_t has been read out.
 // At D = 64 dQ_t has columns of its own.
 //
-// Roles (448 threads):
-//   warps 0-7  dS warps. Thread = key row (TMEM lane) for S^T / dP^T, warps w
-//              and w+4 taking query columns [64 hf, 64 hf + 64). Per step:
-//              exponentials of S^T_t -> P^T_t into TMEM, then dS^T_t into the
-//              shared dS tile.
-//   warp 8     TMA producer: K, V once; Q_t (with the step's LSE and D_i
-//              staged beside it) through a two-stage ring, dO_t through one
-//              stage (dV_t, its last reader, runs long before dP_{t+1}).
-//   warp 9     MMA warp, converged, one elect.sync lane issuing. Order per
-//              step: dP_t, dV_t, S_{t+1}, dQ_t, dK_t. dQ_t goes right after dS_t
-//              because its read-out gates dP_{t+1}; the exponentials of step
-//              t+1 overlap dQ_t and dK_t, and the dS phase of step t overlaps
-//              dV_t and S_{t+1}.
-//   warps 10-13 dQ warps. Thread = query row of dQ_t (TMEM lane): read-out,
-//              staging and reductions, off the dS warps' path, so that the
-//              exponentials of step t+1 run while dQ_t is read out and dP_{t+1}
-//              is formed.
+// Roles (512 threads, four warpgroups):
+//   warps 0-7   dS warps (warpgroups 0, 1; 128 registers). Thread = key row
+//               (TMEM lane) for S^T / dP^T, warps w and w+4 taking query
+//               columns [64 hf, 64 hf + 64). Per step: exponentials of S^T_t
+//               -> P^T_t into TMEM, then dS^T_t into the shared dS tile.
+//   warps 8-11  dQ warps (warpgroup 2; 176 registers, enough to hold a whole
+//               row block of dQ_t). Thread = query row of dQ_t (TMEM lane):
+//               the read-out in one go, dq_free, then the staging and the
+//               reductions, off the dS warps' path. With the read-out this
+//               short, dP_{t+1} follows dQ_t closely and the staging runs
+//               during the exponentials of step t+1 rather than during its
+//               dS phase, whose shared-memory stores it would compete with.
+//   warp 12     TMA producer (warpgroup 3; 80 registers): K, V once; Q_t (with
+//               the step's LSE and D_i staged beside it) through a two-stage
+//               ring, dO_t through one stage (dV_t, its last reader, runs long
+//               before dP_{t+1}).
+//   warp 13     MMA warp (warpgroup 3), converged, one elect.sync lane
+//               issuing. Order per step: dP_t, dV_t, S_{t+1}, dQ_t, dK_t. dQ_t
+//               goes right after dS_t because its read-out gates dP_{t+1}; the
+//               exponentials of step t+1 overlap dQ_t and dK_t, and the dS
+//               phase of step t overlaps dV_t and S_{t+1}.
+//   warps 14-15 no role (they complete warpgroup 3 for its register count).
 #include <limits.h>
 #include <math.h>
 
@@ -65,12 +70,19 @@ namespace {
 namespace fused {
 
 constexpr int BT = 128;        // keys per CTA = query rows per step = TMEM lanes
-constexpr int THREADS = 448;
-constexpr int N_DS = 256;      // dS warps' threads
-constexpr int WARP_TMA = 8;
-constexpr int WARP_MMA = 9;
-constexpr int WARP_DQ0 = 10;   // dQ warps 10-13: TMEM lane quarters 2, 3, 0, 1
+constexpr int THREADS = 512;
+constexpr int N_DS = 256;      // dS warps' threads (warpgroups 0 and 1)
+constexpr int WARP_DQ0 = 8;    // dQ warps 8-11 (warpgroup 2): TMEM lane quarters 0-3
 constexpr int N_DQ = 128;      // dQ warps' threads
+constexpr int WARP_TMA = 12;   // warpgroup 3: producer, MMA warp, two idle warps
+constexpr int WARP_MMA = 13;
+// Registers per thread (setmaxnreg): the block launches at 128 (16 warps,
+// four per SM sub-partition, 16K registers each). Warpgroup 3 gives back 48
+// of them per thread and the dQ warps take them, enough to hold a whole dQ_t
+// row block: 2 x 128 + 176 + 80 = 4 x 128 on every sub-partition and for the
+// block.
+constexpr uint32_t REG_DQ = 176;
+constexpr uint32_t REG_CTRL = 80;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr unsigned FULL = 0xffffffffu;
 constexpr uint32_t SPAN = BT * 128;   // 128 rows x 128 bytes: one 128-byte swizzle column block
@@ -83,7 +95,6 @@ struct Cfg {
   static constexpr int QS = 2;                       // Q stages (with LSE, D_i)
   static constexpr int GS = 1;                       // dO stages (dO_{t+1} is read after dV_t)
   static constexpr bool ALIAS = D == 128;            // dQ_t formed over dP
-  static constexpr int ROUNDS = D / 64;              // dQ read-out rounds of two 32 x 32 boxes
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr uint32_t TM_DQ = ALIAS ? TM_DP : 256 + 2 * D;
   static constexpr uint32_t OFF_K = 0;
@@ -147,6 +158,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
   return __all_sync(FULL, ok);
 }
 
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // One 128-row tile of a token-major tensor (its D / 64 column blocks).
 template <int D>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -206,11 +226,8 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-// 14 warps put four on each of two SM sub-partitions, whose 16K registers
-// then allow 128 per thread: the bound of 512 threads holds the compiler to
-// that.
 template <int D>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -278,6 +295,10 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Each warpgroup sets its register count at the head of its own branch,
+  // so the compiler fits each branch's code to it.
+  if (warp / 4 == WARP_TMA / 4) {
+  regs_dec<REG_CTRL>();
   if (warp == WARP_TMA) {
     // ------------------------------------------------------------ producer ---
     float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -453,13 +474,16 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
     tc_commit_if(leader, bars.dkv_done());
-  } else if (warp >= WARP_DQ0) {
+  }   // warps 14 and 15: no role
+  } else if (warp / 4 == WARP_DQ0 / 4) {
+    regs_inc<REG_DQ>();
     // ------------------------------------------------------------ dQ warps ---
-    // Thread = query row (warp & 3) * 32 + lane of the step's tile. Each
-    // round reads two 32 x 32 boxes of dQ_t (fp32) out of TMEM, stages them
-    // 128-byte swizzled in this warp's 8 KB of the staging area, and one lane
-    // adds them into dQacc with TMA tensor reductions, which run on their own.
-    // dq_free goes out as soon as the last round is in registers.
+    // Thread = query row (warp & 3) * 32 + lane of the step's tile. The
+    // whole row block of dQ_t (D / 32 boxes of 32 x 32 fp32) comes out of
+    // TMEM at once and dq_free goes out; then, two boxes a round, the boxes
+    // are staged 128-byte swizzled in this warp's 8 KB of the staging area
+    // and one lane adds them into dQacc with TMA tensor reductions, which run
+    // on their own.
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t stg = sbase + C::OFF_STG + (warp - WARP_DQ0) * 8192u;
     const bool stamp = warp == WARP_DQ0 && lane == 0;   // debug stamps
@@ -467,6 +491,15 @@ __global__ void __launch_bounds__(512, 1)
       if (!warp_wait(bars.dq_full(), t & 1, p.err, abort, W_DQFULL)) break;
       if (stamp) FA_STAMP(p, T_Q_DQFULL, t);
       tc_fence_after();
+      uint32_t a[D / 32][32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_off + C::TM_DQ + 32 * c, a[c]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) reg_fence(a[c]);
+      tc_fence_before();
+      mbar_arrive(bars.dq_free());
+      if (stamp) FA_STAMP(p, T_Q_DQFREE, t);
       const int h = hk * g + t / n_qt;
       const int row0 = sq.start + (i0 + t % n_qt) * BT + (warp & 3) * 32;
       // Rows past the sequence's end hold exact zeros (their dS rows are
@@ -475,18 +508,7 @@ __global__ void __launch_bounds__(512, 1)
       // sequence is not added at all.
       const bool add = row0 < sq.start + sq.len;
 #pragma unroll
-      for (int rd = 0; rd < C::ROUNDS; ++rd) {
-        uint32_t a[2][32];
-        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * rd, a[0]);
-        tmem_ld32(tmem + lane_off + C::TM_DQ + 64 * rd + 32, a[1]);
-        tmem_ld_wait();
-        reg_fence(a[0]);
-        reg_fence(a[1]);
-        if (rd == C::ROUNDS - 1) {
-          tc_fence_before();
-          mbar_arrive(bars.dq_free());
-          if (stamp) FA_STAMP(p, T_Q_DQFREE, t);
-        }
+      for (int rd = 0; rd < D / 64; ++rd) {
         // The slots' previous boxes must have been read.
         if (lane == 0) bulk_wait_read_all();
         __syncwarp();
@@ -494,8 +516,9 @@ __global__ void __launch_bounds__(512, 1)
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int m = 0; m < 8; ++m)
-            st_shared_v4(stg + c * 4096u + lane * 128 + ((m ^ (lane & 7)) << 4), a[c][4 * m],
-                         a[c][4 * m + 1], a[c][4 * m + 2], a[c][4 * m + 3]);
+            st_shared_v4(stg + c * 4096u + lane * 128 + ((m ^ (lane & 7)) << 4),
+                         a[2 * rd + c][4 * m], a[2 * rd + c][4 * m + 1], a[2 * rd + c][4 * m + 2],
+                         a[2 * rd + c][4 * m + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && add &&
