@@ -128,6 +128,7 @@ KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "decode": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "decode_t": ("decode_t.cu", "decode_t.h", "common.cuh", "params.h"),
                   "fp8_fwd": ("fwd_bf16.cu", "common.cuh", "params.h"),
                   "fp8_quantize_kernel": ("fp8.cu", "common.cuh", "params.h")}
 
@@ -834,6 +835,7 @@ def run_decode(args, w) -> None:
     o = torch.empty_like(q)
     lse = torch.empty((q.shape[0], w.H), device=dev, dtype=torch.float32)
     n_split = fa.decode_num_splits(w.B, w.H_kv, max_len)
+    balanced = fa.decode_balanced(w.D, w.q_len, w.H, w.H_kv)
     ws = torch.empty(max(1, fa.decode_workspace_size(w.B, w.q_len, w.H, w.H_kv, w.D, max_len)),
                      dtype=torch.uint8, device=dev)
     alg_bytes = kv_bytes + 2 * q.numel() * q.element_size() + lse.numel() * 4
@@ -911,25 +913,29 @@ def run_decode(args, w) -> None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": dict(decode_config(w), n_split=n_split,
+        "config": dict(decode_config(w),
+                       partition=("balanced: equal key-tile ranges over one persistent CTA "
+                                  "per SM" if balanced else f"{n_split} splits per sequence"),
                        parallelism=f"replicas{world}" if world > 1 else "none",
                        l2=f"not flushed: every step reads {kv_bytes / 2**20:.0f} MiB of cache "
                           f"> {L2_BYTES >> 20} MiB L2",
                        ranks="each rank its own seeded batch of this shape"),
         "tflops": fl / (call_ms / 1e3) / 1e12,
         "kernel_ms": {"fa_decode (partials + merge)": round(call_ms, 4)},
-        "roofline": {"kernel": "fwd_bf16_kernel<decode> + decode_combine_kernel (one fa_decode)",
+        "roofline": {"kernel": ("decode_t_kernel + decode_t_merge_kernel" if balanced else
+                                "fwd_bf16_kernel<decode> + decode_combine_kernel") +
+                               " (one fa_decode)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peaks['source']} HBM copy",
                      "algorithmic_bytes": alg_bytes,
-                     "traffic": recorded_traffic("decode", w.name)},
+                     "traffic": recorded_traffic("decode_t" if balanced else "decode", w.name)},
         "cpu_baseline": cpu,
         "e2e": {"value": kv_bytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9,
                 "unit": DECODE_UNIT, "steps": e2e_steps, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "how": "public API, pinned host buffers, copies of neighbouring steps "
                        "overlapping the computation (double-buffered, three streams)"},
-        "gpu_launches": (2 if n_split > 1 else 1) * args.steps,
+        "gpu_launches": (2 if balanced or n_split > 1 else 1) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -139,6 +139,13 @@ def decode_num_splits(B: int, H_kv: int, max_seqlen_k: int, n_split: int = 0) ->
     return int(_lib().fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split))
 
 
+def decode_balanced(D: int, q_len: int, H: int, H_kv: int, n_split: int = 0) -> bool:
+    """Whether fa_decode takes its balanced kernel for this shape: automatic
+    splits, D = 128 and at most 64 query rows (q_len x H / H_kv) per kv head
+    (include/fa.h, fa_decode)."""
+    return n_split == 0 and D == 128 and H % H_kv == 0 and q_len * (H // H_kv) <= 64
+
+
 def decode_workspace_size(B: int, q_len: int, H: int, H_kv: int, D: int, max_seqlen_k: int,
                           n_split: int = 0) -> int:
     return int(_lib().fa_decode_workspace_size(B, q_len, H, H_kv, D, max_seqlen_k, n_split))

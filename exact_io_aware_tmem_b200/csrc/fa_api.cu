@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "decode_t.h"
 #include "params.h"
 
 namespace fa {
@@ -251,6 +252,10 @@ int fa_decode_num_splits(int B, int H_kv, int max_seqlen_k, int requested) {
 size_t fa_decode_workspace_size(int B, int q_len, int H, int H_kv, int D, int max_seqlen_k,
                                 int n_split) {
   if (B <= 0 || q_len <= 0 || H <= 0 || H_kv <= 0 || D <= 0 || max_seqlen_k < 0) return 0;
+  if (n_split == 0 && H % H_kv == 0 &&
+      fa::decode_t_eligible(D, static_cast<long long>(q_len) * (H / H_kv)))
+    return fa::decode_t_workspace(B, H_kv, static_cast<long long>(q_len) * (H / H_kv),
+                                  fa::decode_t_ctas());
   const int ns = fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split);
   if (ns <= 1) return 0;
   const size_t rows = static_cast<size_t>(ns) * B * q_len * H;
@@ -313,6 +318,8 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, voi
   p.err.budget = fa::g_budget;
   p.err.word = fa::err_word();
   if (p.err.word == nullptr) return FA_ERR_CUDA;
+  p.trace = fa::g_trace;
+  p.trace_cta = fa::g_trace_cta;
 
   fa::DecodeArgs d = {};
   d.cache_seqlens = cache_seqlens;
@@ -333,6 +340,14 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, voi
                                           fa::round256(rows * D * 4));
   }
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (n_split == 0 && fa::decode_t_eligible(D, d.n_rows)) {
+    // Balanced partition over one persistent CTA per SM (decode_t.cu); the
+    // workspace size above was computed for the same device.
+    fa::DecodeTArgs t = {};
+    t.ctas = fa::decode_t_ctas();
+    fa::decode_t_carve(t, workspace, B, H_kv, d.n_rows);
+    return fa::cuda_status(fa::launch_decode_t(p, d, t, s));
+  }
   return fa::cuda_status(fa::launch_decode_bf16(p, d, s));
 }
 

@@ -10,6 +10,7 @@ what.
 
   python -m exact_io_aware_tmem_b200.trace --kernel bwd --workload NAME [--cta 0]
   python -m exact_io_aware_tmem_b200.trace --kernel fwd --workload NAME
+  python -m exact_io_aware_tmem_b200.trace --kernel dec --workload DECODE_NAME
 
 The traced CTA is blockIdx.x (0: the first launched, with the longest causal
 work).
@@ -32,6 +33,9 @@ FWD_KINDS = {
     "W0_SFULL": 7, "W0_LD": 8, "W0_EXP": 9, "W0_ARR": 10,
     "W1_SFULL": 11, "W1_LD": 12, "W1_EXP": 13, "W1_ARR": 14,
     "M_PREADY0": 15, "M_PREADY1": 16,
+}
+DEC_KINDS = {
+    "P_K": 0, "P_V": 1, "M_S": 2, "M_PV": 3, "W_SFULL": 4, "W_ARR": 5, "W_EPI": 6,
 }
 # (label, from event, step offset of from, to event, step offset of to): the
 # median of stamp[to][t + dto] - stamp[from][t + dfrom] over the steps t.
@@ -87,6 +91,20 @@ FWD_SPANS = [
 ]
 
 
+DEC_SPANS = [
+    ("producer: K_j issued -> S_j issued (K landed, S buffer free)", "P_K", 0, "M_S", 0),
+    ("tensor: S_j issued -> softmax sees S_j", "M_S", 0, "W_SFULL", 0),
+    ("softmax: S_j seen -> P_j published", "W_SFULL", 0, "W_ARR", 0),
+    ("MMA warp: P_j published -> P_j V_j issued", "W_ARR", 0, "M_PV", 0),
+    ("softmax: tile period (P_j -> P_{j+1} published)", "W_ARR", 0, "W_ARR", 1),
+    ("MMA warp: tile period (P_j V_j -> P_{j+1} V_{j+1})", "M_PV", 0, "M_PV", 1),
+    ("producer: K_j issue period", "P_K", 0, "P_K", 1),
+    ("producer: V_j issue period", "P_V", 0, "P_V", 1),
+    ("producer: K_{j+3} issued after S_j issued (slot refill)", "M_S", 0, "P_K", 3),
+    ("producer: V_{j+3} issued after P_j V_j issued (slot refill)", "M_PV", 0, "P_V", 3),
+]
+
+
 def spans(stamps, kinds: dict, table, n_steps: int, skip: int = 2) -> list:
     """(label, median cycles, count) for each span of ``table``."""
     out = []
@@ -103,6 +121,41 @@ def spans(stamps, kinds: dict, table, n_steps: int, skip: int = 2) -> list:
     return out
 
 
+def run_decode(workload: str, cta: int = 0):
+    """Runs fa_decode on the decode workload through the debug build with the
+    partials kernel stamping its events (the balanced kernel's, for the
+    shapes it takes). Returns (stamps, key tiles of the traced CTA)."""
+    import torch
+
+    from . import attention as fa
+    from . import _abi
+    from .workloads import DECODE_WORKLOADS, make_decode_inputs
+
+    w = DECODE_WORKLOADS[workload]
+    inp = make_decode_inputs(w)
+    dev = torch.device("cuda", 0)
+    L = w.lengths()
+    q = inp.q.to(dev)
+    kc = inp.k_cache.to(dev)
+    vc = inp.v_cache.to(dev)
+    lens = inp.cache_seqlens.to(dev)
+    tb = None if inp.block_table is None else inp.block_table.to(dev)
+    args = dict(q_len=w.q_len, max_seqlen_k=max(L), block_table=tb, page_size=inp.page_size,
+                causal=w.causal)
+    buf = torch.zeros(_abi.DEBUG_TRACE_BYTES // 8, dtype=torch.int64, device=dev)
+    with fa.debug_build() as lib:
+        assert lib.fa_debug_build() == 1
+        fa.decode(q, kc, vc, lens, **args)   # warm-up
+        _abi.check(lib.fa_debug_set_trace(buf.data_ptr(), buf.numel() * 8, cta), "trace")
+        fa.decode(q, kc, vc, lens, **args)
+        _abi.check(lib.fa_debug_set_trace(None, 0, 0), "trace")
+        st, where = fa.check_device_error(dev)
+        if st != 0:
+            raise RuntimeError(f"device error {st} at {where:#x}")
+    stamps = buf.view(32, 1024).cpu().numpy()
+    return stamps, int((stamps[DEC_KINDS["M_PV"]] != 0).sum())
+
+
 def run(kernel: str, workload: str, cta: int = 0):
     """Runs the forward (and, for ``bwd``, the backward) of the workload on
     cuda:0 through the debug build with stamping on for the kernel asked
@@ -112,6 +165,9 @@ def run(kernel: str, workload: str, cta: int = 0):
     from . import attention as fa
     from . import _abi
     from .workloads import WORKLOADS, make_inputs
+
+    if kernel == "dec":
+        return run_decode(workload, cta)
 
     w = WORKLOADS[workload]
     inp = make_inputs(w)
@@ -157,14 +213,15 @@ def run(kernel: str, workload: str, cta: int = 0):
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("--kernel", choices=["fwd", "bwd"], required=True)
+    ap.add_argument("--kernel", choices=["fwd", "bwd", "dec"], required=True)
     ap.add_argument("--workload", default="bf16_causal_b2_h16_n8192_d128")
     ap.add_argument("--cta", type=int, default=0)
     args = ap.parse_args(argv)
     from .build import build
     build(debug=True)
     stamps, n = run(args.kernel, args.workload, args.cta)
-    kinds, table = (BWD_KINDS, BWD_SPANS) if args.kernel == "bwd" else (FWD_KINDS, FWD_SPANS)
+    kinds, table = {"bwd": (BWD_KINDS, BWD_SPANS), "fwd": (FWD_KINDS, FWD_SPANS),
+                    "dec": (DEC_KINDS, DEC_SPANS)}[args.kernel]
     print(f"{args.kernel} {args.workload} CTA {args.cta}: {n} steps stamped; median cycles "
           f"over the steady-state steps")
     for label, med, cnt in spans(stamps, kinds, table, n):

@@ -185,6 +185,25 @@ def test_decode_split_count_and_workspace_size(lib):
         r256(rows * 4)
 
 
+def test_balanced_decode_workspace_size(lib):
+    # Automatic splits at D = 128 with q_len * g <= 64 take the balanced
+    # kernel: partial rows for (B * H_kv + CTAs) slots, plus two int arrays
+    # of B * H_kv. Without a device the library assumes 148 CTAs (B200 SMs).
+    def r256(x):
+        return (x + 255) // 256 * 256
+    for B, q_len, H, H_kv in [(16, 1, 32, 8), (16, 8, 32, 8), (3, 16, 16, 4)]:
+        segs = B * H_kv
+        rows = (segs + 148) * q_len * (H // H_kv)
+        want = r256(rows * 128 * 4) + r256(rows * 4) + 2 * r256(segs * 4)
+        assert lib.fa_decode_workspace_size(B, q_len, H, H_kv, 128, 32768, 0) == want
+    # more than 64 rows (16 tokens x 8 heads), or an explicit split count:
+    # the split kernel's partials
+    rows = lib.fa_decode_num_splits(2, 2, 1000, 0) * 2 * 16 * 16
+    assert lib.fa_decode_workspace_size(2, 16, 16, 2, 128, 1000, 0) == \
+        r256(rows * 128 * 4) + r256(rows * 4)
+    assert lib.fa_decode_workspace_size(2, 1, 8, 2, 128, 1000, 1) == 0
+
+
 # --------------------------------------------------------------------- FP8 ---
 
 def test_fp8_entry_points_reject_bad_shapes(lib):

@@ -101,6 +101,63 @@ def test_many_splits_and_scale():
     _check(o, lse, *_ref(c, causal=True, scale=0.2))
 
 
+# Balanced decode (D = 128, q_len * g <= 64, automatic splits): one persistent
+# CTA per SM over equal ranges of (sequence, kv head, key tile) units.
+BALANCED_LENGTHS = [1, 127, 128, 129, 0, 1000, 255, 256, 3000, 40, 2049, 7]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("q_len,H,H_kv", [(1, 8, 2), (3, 15, 3), (5, 16, 4), (8, 32, 8),
+                                          (16, 16, 4), (9, 21, 3)])
+def test_balanced_rows_and_lengths(q_len, H, H_kv, causal):
+    # R = q_len * g = 4, 15, 20, 32, 64, 63: the 16-, 32- and 64-column
+    # forms, odd g, and rows that do not fill their column block.
+    c = decode_case(71 + q_len * H, dtype="bf16", lengths=BALANCED_LENGTHS, q_len=q_len, H=H,
+                    H_kv=H_kv, D=128)
+    o, lse = _run(c, causal=causal, n_split=0)
+    _check(o, lse, *_ref(c, causal=causal, scale=128 ** -0.5))
+
+
+@pytest.mark.parametrize("page", [16, 64, 128, 256])
+def test_balanced_paged(page):
+    c = decode_case(81 + page, dtype="bf16", lengths=BALANCED_LENGTHS, q_len=2, H=8, H_kv=2,
+                    D=128, page_size=page)
+    o, lse = _run(c, causal=True, n_split=0)
+    _check(o, lse, *_ref(c, causal=True, scale=128 ** -0.5))
+
+
+def test_balanced_more_ctas_than_tiles():
+    # 6 tiles over one CTA per SM: most ranges are empty, some of them
+    # strictly inside a segment whose pieces lie on both sides.
+    c = decode_case(91, dtype="bf16", lengths=[300, 5, 0, 390], q_len=1, H=4, H_kv=1, D=128)
+    o, lse = _run(c, causal=True, n_split=0)
+    _check(o, lse, *_ref(c, causal=True, scale=128 ** -0.5))
+
+
+def test_balanced_many_sequences():
+    # 96 sequences: each CTA's range crosses several segments (Q buffers
+    # reused, pieces written whole and as partials).
+    rng = np.random.default_rng(17)
+    lengths = [int(x) for x in rng.integers(0, 1500, size=96)]
+    c = decode_case(101, dtype="bf16", lengths=lengths, q_len=1, H=16, H_kv=4, D=128)
+    o, lse = _run(c, causal=True, n_split=0)
+    _check(o, lse, *_ref(c, causal=True, scale=128 ** -0.5))
+
+
+def test_balanced_reference_moves_mid_piece():
+    # Keys whose norm grows along the cache: later tiles exceed the running
+    # reference by far more than 2^8, so it moves inside pieces and O^T is
+    # rescaled in TMEM.
+    lengths = [5000, 2600, 900]
+    c = decode_case(111, dtype="bf16", lengths=lengths, q_len=2, H=8, H_kv=2, D=128)
+    ramp = torch.ones(c.k_cache.shape[0])
+    for b, n in enumerate(lengths):
+        ramp[b * c.page_size:b * c.page_size + n] = 1 + torch.arange(n) / 1024.0
+    c.k_cache = (c.k_cache.float() * ramp[:, None, None]).to(c.k_cache.dtype)
+    o, lse = _run(c, causal=True, n_split=0, scale=0.5)
+    _check(o, lse, *_ref(c, causal=True, scale=0.5))
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name", sorted(DECODE_WORKLOADS))
 def test_decode_workload_sampled(name):
