@@ -51,9 +51,10 @@ constexpr int D = 128;
 constexpr int BN = 128;                   // keys per tile
 constexpr int CHUNKS = D / 64;            // 128-byte column blocks of a bf16 row
 constexpr int STAGES = 3;
-constexpr int THREADS = 192;
-constexpr int WARP_TMA = 4;
-constexpr int WARP_MMA = 5;
+constexpr int SOFTMAX_THREADS = 256;
+constexpr int THREADS = SOFTMAX_THREADS + 64;
+constexpr int WARP_TMA = 8;
+constexpr int WARP_MMA = 9;
 constexpr uint32_t KV_SPAN = BN * 128;    // one column block of a K / V tile
 constexpr uint32_t TILE = BN * D * 2;     // K / V tile
 constexpr float RESCALE_LOG2 = 8.f;
@@ -74,8 +75,7 @@ struct Cfg {
   static constexpr uint32_t OFF_MREF = OFF_P + PBUF * QP_BYTES;  // float [NQ]: reference max
   static constexpr uint32_t OFF_ALPHA = OFF_MREF + NQ * 4;    // float [NQ]: its last move
   static constexpr uint32_t OFF_RED = OFF_ALPHA + NQ * 4;     // float [4][NQ]: per-warp max / sum
-  static constexpr uint32_t OFF_FLAG = OFF_RED + 4 * NQ * 4;  // int [2][4]: per-warp "moves"
-  static constexpr uint32_t OFF_ROWS = OFF_FLAG + 32;        // int [8][8]: paged rows per tile
+  static constexpr uint32_t OFF_ROWS = OFF_RED + 4 * NQ * 4;  // int [8][8]: paged rows per tile
   static constexpr uint32_t OFF_BAR = OFF_ROWS + 8 * 8 * 4;
   // k_full[S], k_empty[S], v_full[S], v_empty[S], q_full[QBUF], q_empty[QBUF],
   // s_full[2], s_free[2], p_ready[PBUF], pv_done[PBUF], v_land
@@ -145,22 +145,36 @@ __device__ __forceinline__ bool warp_test(uint32_t bar, uint32_t parity) {
   return __all_sync(FULL, done != 0);
 }
 
-// The four softmax warps (128 threads) meet at named barrier 1. The AND form
-// also tells every thread whether all of them are still on track, so that a
-// failed wait in one warp ends the loop of all four at the same barrier.
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The eight softmax warps (256 threads) meet at named barrier 1. The AND
+// form also tells every thread whether all of them are still on track, so
+// that a failed wait in one warp ends the loop of all eight at the same
+// barrier; the OR form gathers a vote.
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ bool softmax_sync_and(bool ok) {
   uint32_t all;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(all)
       : "r"(ok ? 1u : 0u)
       : "memory");
   return all != 0;
+}
+
+__device__ __forceinline__ bool softmax_sync_or(bool v) {
+  uint32_t any;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(any)
+      : "r"(v ? 1u : 0u)
+      : "memory");
+  return any != 0;
 }
 
 // 32 lanes x 16 consecutive 32-bit TMEM columns.
@@ -184,21 +198,45 @@ __device__ __forceinline__ void tmem_st16p(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// NQ consecutive columns of this thread's TMEM lane (16 at a time), valid
-// on return.
-template <int NQ>
-__device__ __forceinline__ void tmem_row_ld(uint32_t taddr, uint32_t (&r)[NQ]) {
-#pragma unroll
-  for (int c = 0; c < NQ / 16; ++c) tmem_ld16(taddr + 16 * c, r + 16 * c);
-  tmem_ld_wait();
-#pragma unroll
-  for (int i = 0; i < NQ; ++i) asm volatile("" : "+r"(r[i]));
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
 }
 
-template <int NQ>
-__device__ __forceinline__ void tmem_row_st(uint32_t taddr, const uint32_t (&r)[NQ]) {
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+// N (8, 16, 32) consecutive columns of this thread's TMEM lane, valid on
+// return.
+template <int N>
+__device__ __forceinline__ void tmem_row_ld(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 8) {
+    tmem_ld8(taddr, r);
+  } else {
 #pragma unroll
-  for (int c = 0; c < NQ / 16; ++c) tmem_st16p(taddr + 16 * c, r + 16 * c);
+    for (int c = 0; c < N / 16; ++c) tmem_ld16(taddr + 16 * c, r + 16 * c);
+  }
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_row_st(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 8) {
+    tmem_st8(taddr, r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < N / 16; ++c) tmem_st16p(taddr + 16 * c, r + 16 * c);
+  }
   tmem_st_wait();
 }
 
@@ -218,7 +256,7 @@ __host__ __device__ __forceinline__ int seq_tiles(const int* lens, int b, int ma
 // Position of a role in the CTA's range of units: key tile t of kv head hk of
 // sequence b, unit u. Every role walks the same sequence of tiles.
 struct Walk {
-  int b, hk, t;
+  int b, t;
   int n, len;               // tiles and keys of sequence b
   long long u, u0, u1;      // current unit, the CTA's range [u0, u1)
   __host__ __device__ bool done() const { return u >= u1; }
@@ -226,13 +264,11 @@ struct Walk {
   __host__ __device__ bool first() const { return t == 0 || u == u0; }
   __host__ __device__ bool last() const { return t + 1 == n || u + 1 == u1; }
   __host__ __device__ bool seg_end() const { return t + 1 == n; }
-  __host__ __device__ void next(const int* lens, int B, int H_kv, int max_len) {
+  __host__ __device__ void next(const int* lens, int B, int max_len) {
     ++u;
     ++t;
     if (u >= u1 || t < n) return;
     t = 0;
-    if (++hk < H_kv) return;
-    hk = 0;
     do {
       if (++b >= B) {
         u = u1;
@@ -242,11 +278,11 @@ struct Walk {
     } while (n == 0);
   }
   // To the first tile of the next piece.
-  __host__ __device__ void next_piece(const int* lens, int B, int H_kv, int max_len) {
+  __host__ __device__ void next_piece(const int* lens, int B, int max_len) {
     const long long step = (n - t < u1 - u) ? static_cast<long long>(n - t) : u1 - u;
     u += step - 1;
     t += static_cast<int>(step - 1);
-    next(lens, B, H_kv, max_len);
+    next(lens, B, max_len);
   }
 };
 
@@ -285,18 +321,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
-      mbar_init(bars.s_free(i), 128);
+      mbar_init(bars.s_free(i), SOFTMAX_THREADS);
     }
     for (int i = 0; i < C::PBUF; ++i) {
-      mbar_init(bars.p_ready(i), 128);
+      mbar_init(bars.p_ready(i), SOFTMAX_THREADS);
       mbar_init(bars.pv_done(i), 1);
     }
     mbar_init(bars.v_land(), 1);
     fence_mbar_init();
   }
+  // CTA c serves kv head c % H_kv over range c / H_kv of the groups.
+  const int groups = dt.ctas / p.H_kv;
+  const int grp = blockIdx.x / p.H_kv;
+  const int hk = blockIdx.x % p.H_kv;
   if (warp == WARP_TMA) {
-    // This CTA's range [u0, u1) of the U = H_kv * sum_b n_b units, and the
-    // tile at u0: a scan of the lengths, 32 sequences per step.
+    // This CTA's range [u0, u1) of the U = sum_b n_b units, and the tile at
+    // u0: a scan of the lengths, 32 sequences per step.
     long long tot = 0;
     for (int b0 = 0; b0 < p.B; b0 += 32) {
       const int b = b0 + lane;
@@ -309,9 +349,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 #pragma unroll
     for (int sh = 16; sh > 0; sh >>= 1) tot += __shfl_xor_sync(FULL, tot, sh);
-    tot *= p.H_kv;
-    const long long u0 = tot * blockIdx.x / dt.ctas;
-    const long long u1 = tot * (blockIdx.x + 1) / dt.ctas;
+    const long long u0 = tot * grp / groups;
+    const long long u1 = tot * (grp + 1) / groups;
     int sb = 0;
     long long base = 0;
     if (u0 < tot) {
@@ -319,9 +358,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int b0 = 0; b0 < p.B; b0 += 32) {
         const int b = b0 + lane;
         int len = 0;
-        const long long units =
-            (b < p.B) ? static_cast<long long>(seq_tiles(lens, b, p.max_seqlen, len)) * p.H_kv
-                      : 0;
+        const long long units = (b < p.B) ? seq_tiles(lens, b, p.max_seqlen, len) : 0;
         long long incl = units;
 #pragma unroll
         for (int sh = 1; sh < 32; sh <<= 1) {
@@ -340,22 +377,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         acc = __shfl_sync(FULL, incl, 31);
       }
     }
-    int len = 0;
-    const int n = (u0 < tot) ? seq_tiles(lens, sb, p.max_seqlen, len) : 1;
-    const long long off = u0 - base;
+    const long long off = u0 - base;   // < n_sb when u0 < tot
     if (lane == 0) {
       start[0] = sb;
-      start[1] = static_cast<int>(off / n);
-      start[2] = static_cast<int>(off % n);
+      start[1] = static_cast<int>(u0 < tot ? off : 0);
       range[0] = u0;
       range[1] = u1;
     }
-    if (u0 == u1 && u0 < tot && off % n != 0) {
-      // An empty range strictly inside a segment (more CTAs than units):
+    if (u0 == u1 && u0 < tot && off != 0) {
+      // An empty range strictly inside a segment (more groups than tiles):
       // the segment's pieces lie on both sides, so the merge reads this
       // CTA's slot too. It holds no key: LSE -inf.
-      const size_t slot =
-          static_cast<size_t>(sb * p.H_kv + static_cast<int>(off / n) + blockIdx.x) * R;
+      const size_t slot = static_cast<size_t>((sb + grp) * p.H_kv + hk) * R;
       for (int r = lane; r < R; r += 32) dt.lse_part[slot + r] = -INFINITY;
     }
   }
@@ -363,21 +396,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  // Q rows R .. NQ - 1 are never loaded: zero, so that the score columns of
+  // the rows past R are exactly 0 and need no mask.
+  for (int k = threadIdx.x; k < C::QBUF * CHUNKS * (NQ - R) * 8; k += THREADS) {
+    const int unit = k % 8, row = R + (k / 8) % (NQ - R), blk = k / (8 * (NQ - R));
+    *reinterpret_cast<uint4*>(smem + C::OFF_Q + blk * C::SPAN + row * 128 + unit * 16) =
+        make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   Walk w0;
   w0.b = start[0];
-  w0.hk = start[1];
-  w0.t = start[2];
+  w0.t = start[1];
   w0.u0 = range[0];
   w0.u1 = range[1];
   w0.u = w0.u0;
   w0.n = 0;
   w0.len = 0;
   if (w0.u0 < w0.u1) w0.n = seq_tiles(lens, w0.b, p.max_seqlen, w0.len);
-  auto advance = [&](Walk& w) { w.next(lens, p.B, p.H_kv, p.max_seqlen); };
+  auto advance = [&](Walk& w) { w.next(lens, p.B, p.max_seqlen); };
 
   if (warp == WARP_TMA) {
     // ------------------------------------------------------------ producer ---
@@ -437,7 +477,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int row = w.b * dec.page + w.t * BN;
 #pragma unroll
           for (int c = 0; c < CHUNKS; ++c)
-            tma_load_2d(dst + c * KV_SPAN, map, bar, w.hk * D + c * 64, row);
+            tma_load_2d(dst + c * KV_SPAN, map, bar, hk * D + c * 64, row);
         }
       } else {
         int row;
@@ -450,7 +490,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane < n_box) {
 #pragma unroll
           for (int c = 0; c < CHUNKS; ++c)
-            tma_load_2d(dst + c * KV_SPAN + lane * box * 128, map, bar, w.hk * D + c * 64, row);
+            tma_load_2d(dst + c * KV_SPAN + lane * box * 128, map, bar, hk * D + c * 64, row);
         }
       }
     };
@@ -475,10 +515,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int c = 0; c < CHUNKS; ++c)
               tma_load_3d(sbase + C::OFF_Q + qb * C::QP_BYTES + c * C::SPAN, &tm_q,
-                          bars.q_full(qb), c * 64, qw.hk * dec.g, qw.b * dec.q_len);
+                          bars.q_full(qb), c * 64, hk * dec.g, qw.b * dec.q_len);
           }
           ++pq;
-          qw.next_piece(lens, p.B, p.H_kv, p.max_seqlen);
+          qw.next_piece(lens, p.B, p.max_seqlen);
           progress = true;
         }
       }
@@ -551,8 +591,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = false;
         break;
       }
-      __nanosleep(20);   // leave the issue slots to the softmax warp sharing this SMSP
-    }
+          }
     if (ok && lane == 0) {
       // Drain: the tensor core's last arrivals on the empty barriers must
       // land before the CTA's shared memory is released.
@@ -646,37 +685,70 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         break;
       }
-      __nanosleep(20);   // leave the issue slots to the softmax warp sharing this SMSP
-    }
+          }
   } else {
     // ------------------------------------------------------------- softmax ---
-    const int tid = threadIdx.x;   // key of the tile; O^T row at the end of a piece
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // Warp w owns TMEM lanes 32 (w % 4) .. +31 (keys of a tile; rows of O^T
+    // at the end of a piece) and query rows [NH (w / 4), NH (w / 4 + 1)).
+    constexpr int NH = NQ / 2;
+    const int sid = threadIdx.x;                 // 0 .. 255
+    const int quarter = warp & 3;
+    const int kt = quarter * 32 + lane;          // key of the tile / row d of O^T
+    const int r0 = (warp >> 2) * NH;             // this thread's first query row
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     float* mref = reinterpret_cast<float*>(smem + C::OFF_MREF);
     float* alpha_s = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
-    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
-    int* flag = reinterpret_cast<int*>(smem + C::OFF_FLAG);
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);   // [quarter][row]
     const float c2 = p.scale_log2;
     const int g = dec.g;
-    // This thread's P word for a row pair holds keys (tid & ~1, tid | 1) of
+    // This thread's P word for a row pair holds keys (kt & ~1, kt | 1) of
     // row r (even thread) or r + 1 (odd thread): the pair's column block,
     // 16-byte unit (swizzled by the row below) and byte in the unit.
-    const int kp = tid & ~1;
+    const int kp = kt & ~1;
     const uint32_t p_chunk = C::OFF_P + (kp >> 6) * C::SPAN;
     const int p_unit = (kp & 63) >> 3;
     const int p_byte = (kp & 7) * 2;
-    const bool odd = (tid & 1) != 0;
-    // Rows past R: reference 0 and no move, so their P is 2^-inf = 0 and the
-    // per-row loops below run over all NQ rows without a branch.
-    for (int r = tid; r < NQ; r += 128) {
-      mref[r] = 0.f;
-      alpha_s[r] = 1.f;
+    const bool odd = (lane & 1) != 0;
+    // Rows past R: scores 0 (zero Q rows) or -inf (masked), reference +inf
+    // and no move, so their P is 2^-inf = 0 and the per-row loops below run
+    // over all of this thread's rows without a branch.
+    if (sid < NQ) {
+      mref[sid] = sid < R ? 0.f : INFINITY;
+      alpha_s[sid] = 1.f;
     }
     softmax_sync();
-    Walk w = w0;
-    float l[NQ];   // this thread's part of each row sum, in the current reference
+    // This thread's rows' references: the move threshold m + 8 and the
+    // exponent offset (0 while a row has seen no key, m = -inf), kept in
+    // registers up to 16 rows a thread, read from shared memory beyond.
+    constexpr bool REF_REGS = NH <= 16;
+    float mt[REF_REGS ? NH : 1], mu[REF_REGS ? NH : 1];
+    auto load_ref = [&]() {
+      if constexpr (REF_REGS) {
 #pragma unroll
-    for (int r = 0; r < NQ; ++r) l[r] = 0.f;
+        for (int r = 0; r < NH; ++r) {
+          const float m = mref[r0 + r];
+          mt[r] = m + RESCALE_LOG2;
+          mu[r] = (m == -INFINITY) ? 0.f : m;
+        }
+      }
+    };
+    auto thr = [&](int r) -> float {
+      if constexpr (REF_REGS) return mt[r];
+      else return mref[r0 + r] + RESCALE_LOG2;
+    };
+    auto off = [&](int r) -> float {
+      if constexpr (REF_REGS) {
+        return mu[r];
+      } else {
+        const float m = mref[r0 + r];
+        return (m == -INFINITY) ? 0.f : m;
+      }
+    };
+    load_ref();
+    Walk w = w0;
+    float l[NH];   // this thread's part of its rows' sums, in the current reference
+#pragma unroll
+    for (int r = 0; r < NH; ++r) l[r] = 0.f;
     int i = 0;     // the CTA's tile counter
     int t0 = 0;    // first tile of the current piece
     bool ok = true;
@@ -686,82 +758,86 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (first) {
         t0 = w.t;
 #pragma unroll
-        for (int r = 0; r < NQ; ++r) l[r] = 0.f;
+        for (int r = 0; r < NH; ++r) l[r] = 0.f;
       }
-      uint32_t s[NQ];
+      uint32_t s[NH];
       ok = ok && warp_wait(bars.s_full(i & 1), (i >> 1) & 1, p.err, abort, W_SFULL);
       if (ok) {
         if (warp == 0 && lane == 0) FA_STAMP(p, T_W_SFULL, i);
         tc_fence_after();
-        tmem_row_ld<NQ>(tmem + lane_off + C::TM_S + (i & 1) * NQ, s);
+        tmem_row_ld<NH>(tmem + lane_off + C::TM_S + (i & 1) * NQ + r0, s);
         tc_fence_before();
         mbar_arrive(bars.s_free(i & 1));
       }
       // Query row r sees key `key` when key < len and, causally, key <=
-      // len - q_len + r / g, i.e. r >= g * (key - len + q_len).
-      const int key = w.t * BN + tid;
-      const int rmin = p.causal ? max(0, g * (key - (w.len - dec.q_len))) : 0;
-      const int rlim = key < w.len ? R : 0;
-      float x[NQ];
-      bool ex = false;
+      // len - q_len + r / g, i.e. r >= g * (key - len + q_len). Only a tile
+      // that reaches past len - q_len (causal) or len - 1 needs the mask.
+      float x[NH];
+      if ((w.t + 1) * BN <= (p.causal ? w.len - dec.q_len + 1 : w.len)) {
 #pragma unroll
-      for (int r = 0; r < NQ; ++r)
-        x[r] = (r >= rmin && r < rlim) ? __uint_as_float(s[r]) * c2 : -INFINITY;
+        for (int r = 0; r < NH; ++r) x[r] = __uint_as_float(s[r]) * c2;
+      } else {
+        const int key = w.t * BN + kt;
+        const int rmin = p.causal ? max(0, g * (key - (w.len - dec.q_len))) : 0;
+        const int rlim = key < w.len ? R : 0;
+#pragma unroll
+        for (int r = 0; r < NH; ++r)
+          x[r] = (r0 + r >= rmin && r0 + r < rlim) ? __uint_as_float(s[r]) * c2 : -INFINITY;
+      }
+      bool ex = false;
       if (!first) {
 #pragma unroll
-        for (int r = 0; r < NQ; ++r) ex |= x[r] > mref[r] + RESCALE_LOG2;
+        for (int r = 0; r < NH; ++r) ex |= x[r] > thr(r);
       }
-      // Does any score move its row's reference? One word per warp, two sets
-      // by tile parity.
-      const bool wex = __any_sync(FULL, ex);
-      if (lane == 0) flag[(i & 1) * 4 + warp] = wex ? 1 : 0;
-      if (!softmax_sync_and(ok)) break;
-      const int* fl = flag + (i & 1) * 4;
-      const bool move = first || (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
+      // Does any score move its row's reference (or has a wait failed)? The
+      // rare yes takes a second barrier that tells the two apart.
+      const bool any = softmax_sync_or(ex || !ok);
+      if (any && !softmax_sync_and(ok)) break;
+      const bool move = first || any;
       bool rescale = false;
       if (move) {
         // Row maxima over the 128 keys: per warp by shuffles, then thread r
-        // combines the four warps and moves row r's reference.
+        // combines the four quarters and moves row r's reference.
 #pragma unroll
-        for (int r = 0; r < NQ; ++r) {
-          if (r < R) {
+        for (int r = 0; r < NH; ++r) {
+          if (r0 + r < R) {
             float v = x[r];
 #pragma unroll
             for (int sh = 16; sh > 0; sh >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, sh));
-            if (lane == 0) red[warp * NQ + r] = v;
+            if (lane == 0) red[quarter * NQ + r0 + r] = v;
           }
         }
         softmax_sync();
-        if (tid < R) {
-          const float tmax = fmaxf(fmaxf(red[tid], red[NQ + tid]),
-                                   fmaxf(red[2 * NQ + tid], red[3 * NQ + tid]));
-          const float mo = first ? -INFINITY : mref[tid];
+        if (sid < R) {
+          const float tmax = fmaxf(fmaxf(red[sid], red[NQ + sid]),
+                                   fmaxf(red[2 * NQ + sid], red[3 * NQ + sid]));
+          const float mo = first ? -INFINITY : mref[sid];
           float mn = mo, a = 1.f;
           if (tmax > mo + RESCALE_LOG2) {
             mn = tmax;
             a = (mo == -INFINITY) ? 0.f : ex2_approx(mo - tmax);
           }
-          mref[tid] = mn;
-          alpha_s[tid] = a;
+          mref[sid] = mn;
+          alpha_s[sid] = a;
         }
         softmax_sync();
+        load_ref();
         if (!first) {
 #pragma unroll
-          for (int r = 0; r < NQ; ++r) {
-            const float a = alpha_s[r];
+          for (int r = 0; r < NH; ++r) {
+            const float a = alpha_s[r0 + r];
             l[r] *= a;
             rescale |= a != 1.f;
           }
         }
       }
-      // P = 2^(x - m) for this key and each query row; adjacent keys' values
-      // are paired into one bf16x2 word per row by a shuffle.
-      uint32_t pk[NQ / 2];
+      // P = 2^(x - m) for this key and each of its rows; adjacent keys'
+      // values are paired into one bf16x2 word per row by a shuffle.
+      uint32_t pk[NH / 2];
 #pragma unroll
-      for (int r = 0; r < NQ; r += 2) {
-        const float m0 = mref[r], m1 = mref[r + 1];
-        const float p0 = ex2_approx(x[r] - (m0 == -INFINITY ? 0.f : m0));
-        const float p1 = ex2_approx(x[r + 1] - (m1 == -INFINITY ? 0.f : m1));
+      for (int r = 0; r < NH; r += 2) {
+        const float p0 = ex2_approx(x[r] - off(r));
+        const float p1 = ex2_approx(x[r + 1] - off(r + 1));
         l[r] += p0;
         l[r + 1] += p1;
         const float recv = __shfl_xor_sync(FULL, odd ? p0 : p1, 1);
@@ -780,19 +856,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         uint8_t* pbase = smem + p_chunk + pb * C::QP_BYTES;
 #pragma unroll
-        for (int r = 0; r < NQ; r += 2) {
-          const int row = odd ? r + 1 : r;
+        for (int r = 0; r < NH; r += 2) {
+          const int row = r0 + (odd ? r + 1 : r);
           *reinterpret_cast<uint32_t*>(pbase + row * 128 + ((p_unit ^ (row & 7)) << 4) + p_byte) =
               pk[r >> 1];
         }
         if (rescale) {
-          // Row tid of O^T: column r moves to row r's new reference.
-          uint32_t o[NQ];
-          tmem_row_ld<NQ>(tmem + lane_off + C::TM_O, o);
+          // Row kt of O^T, this thread's columns: column r moves to row r's
+          // new reference.
+          uint32_t o[NH];
+          tmem_row_ld<NH>(tmem + lane_off + C::TM_O + r0, o);
 #pragma unroll
-          for (int r = 0; r < NQ; ++r)
-            o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha_s[r]);
-          tmem_row_st<NQ>(tmem + lane_off + C::TM_O, o);
+          for (int r = 0; r < NH; ++r)
+            o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha_s[r0 + r]);
+          tmem_row_st<NH>(tmem + lane_off + C::TM_O + r0, o);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -805,54 +882,55 @@ __global__ void __launch_bounds__(THREADS, 1)
         // final output when the piece is the whole segment, else as a
         // partial for the merge.
 #pragma unroll
-        for (int r = 0; r < NQ; ++r) {
-          if (r < R) {
+        for (int r = 0; r < NH; ++r) {
+          if (r0 + r < R) {
             float v = l[r];
 #pragma unroll
             for (int sh = 16; sh > 0; sh >>= 1) v += __shfl_xor_sync(FULL, v, sh);
-            if (lane == 0) red[warp * NQ + r] = v;
+            if (lane == 0) red[quarter * NQ + r0 + r] = v;
           }
         }
         if (!softmax_sync_and(ok)) break;
         ok = warp_wait(bars.pv_done(i % C::PBUF), (i / C::PBUF) & 1, p.err, abort, W_PVDONE);
         if (ok) {
           tc_fence_after();
-          uint32_t o[NQ];
-          tmem_row_ld<NQ>(tmem + lane_off + C::TM_O, o);
+          uint32_t o[NH];
+          tmem_row_ld<NH>(tmem + lane_off + C::TM_O + r0, o);
           tc_fence_before();
-          const int seg = w.b * p.H_kv + w.hk;
+          const int seg = w.b * p.H_kv + hk;
           const bool whole = t0 == 0 && w.seg_end();
-          const size_t slot = static_cast<size_t>(seg + blockIdx.x) * R;
+          const size_t slot = static_cast<size_t>((w.b + grp) * p.H_kv + hk) * R;
 #pragma unroll
-          for (int r = 0; r < NQ; ++r) {
+          for (int rr = 0; rr < NH; ++rr) {
+            const int r = r0 + rr;
             if (r < R) {
               const float lt = (red[r] + red[NQ + r]) + (red[2 * NQ + r] + red[3 * NQ + r]);
-              const float v = __uint_as_float(o[r]) * (lt > 0.f ? 1.f / lt : 0.f);
+              const float v = __uint_as_float(o[rr]) * (lt > 0.f ? 1.f / lt : 0.f);
               if (whole) {
                 const size_t orow = static_cast<size_t>(w.b * dec.q_len + r / g) * p.H +
-                                    w.hk * g + r % g;
-                static_cast<__nv_bfloat16*>(p.o)[orow * D + tid] = __float2bfloat16_rn(v);
+                                    hk * g + r % g;
+                static_cast<__nv_bfloat16*>(p.o)[orow * D + kt] = __float2bfloat16_rn(v);
               } else {
-                dt.o_part[(slot + r) * D + tid] = v;
+                dt.o_part[(slot + r) * D + kt] = v;
               }
             }
           }
-          if (tid < R) {
+          if (sid < R) {
             const float lt =
-                (red[tid] + red[NQ + tid]) + (red[2 * NQ + tid] + red[3 * NQ + tid]);
+                (red[sid] + red[NQ + sid]) + (red[2 * NQ + sid] + red[3 * NQ + sid]);
             const float lse =
-                (lt > 0.f) ? (mref[tid] + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+                (lt > 0.f) ? (mref[sid] + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
             if (whole) {
-              const size_t orow = static_cast<size_t>(w.b * dec.q_len + tid / g) * p.H +
-                                  w.hk * g + tid % g;
+              const size_t orow = static_cast<size_t>(w.b * dec.q_len + sid / g) * p.H +
+                                  hk * g + sid % g;
               p.lse[orow] = lse;
             } else {
-              dt.lse_part[slot + tid] = lse;
+              dt.lse_part[slot + sid] = lse;
             }
           }
-          if (tid == 0) {
-            if (t0 == 0) dt.seg_first[seg] = blockIdx.x;
-            if (w.seg_end()) dt.seg_last[seg] = blockIdx.x;
+          if (sid == 0) {
+            if (t0 == 0) dt.seg_first[seg] = grp;
+            if (w.seg_end()) dt.seg_last[seg] = grp;
           }
           if (warp == 0 && lane == 0) FA_STAMP(p, T_W_EPI, i);
         }
@@ -900,17 +978,18 @@ __global__ void __launch_bounds__(256)
     const int c0 = dt.seg_first[seg];
     const int c1 = dt.seg_last[seg];
     if (c0 == c1) return;   // one piece: its CTA wrote the row
-    if (c0 < 0 || c1 >= dt.ctas || c0 > c1) {
+    if (c0 < 0 || c1 >= dt.ctas / p.H_kv || c0 > c1) {
       if (lane == 0) record(p.err, BAD_MERGE);
       return;
     }
+    // Group c's piece of the segment sits in slot (b + c) H_kv + hk.
     for (int c = c0 + lane; c <= c1; c += 32)
-      m = fmaxf(m, dt.lse_part[static_cast<size_t>(seg + c) * R + r]);
+      m = fmaxf(m, dt.lse_part[static_cast<size_t>((b + c) * p.H_kv + hk) * R + r]);
 #pragma unroll
     for (int sh = 16; sh > 0; sh >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, sh));
     if (m != -INFINITY) {
       for (int c = c0; c <= c1; ++c) {
-        const size_t prow = static_cast<size_t>(seg + c) * R + r;
+        const size_t prow = static_cast<size_t>((b + c) * p.H_kv + hk) * R + r;
         const float ls = dt.lse_part[prow];
         if (ls == -INFINITY) continue;
         const float wgt = expf(ls - m);
@@ -947,15 +1026,16 @@ cudaError_t launch_nq(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
 }  // namespace dect
 }  // namespace
 
-int decode_t_ctas() {
+int decode_t_ctas(int H_kv) {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       sms <= 0) {
     cudaGetLastError();
-    return 148;
+    sms = 148;
   }
-  return sms;
+  const int groups = (H_kv > 0 && sms >= H_kv) ? sms / H_kv : 1;
+  return groups * (H_kv > 0 ? H_kv : 1);
 }
 
 size_t decode_t_workspace(long long B, int H_kv, long long n_rows, int ctas) {
@@ -982,7 +1062,9 @@ void decode_t_carve(DecodeTArgs& t, void* workspace, long long B, int H_kv, long
 cudaError_t launch_decode_t(const AttnParams& p, const DecodeArgs& d, const DecodeTArgs& t,
                             cudaStream_t stream) {
   using namespace dect;
-  if (p.D != D || d.n_rows < 1 || d.n_rows > 64 || t.ctas <= 0) return cudaErrorInvalidValue;
+  if (p.D != D || d.n_rows < 1 || d.n_rows > 64 || p.H_kv <= 0 || t.ctas <= 0 ||
+      t.ctas % p.H_kv != 0)
+    return cudaErrorInvalidValue;
   const long long segs = static_cast<long long>(p.B) * p.H_kv;
   if (segs == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;

@@ -8,16 +8,18 @@
 
 namespace fa {
 
-// The U = H_kv * sum_b ceil(len_b / 128) units (sequence b, kv head, 128-key
-// tile), taken in that order, are cut into ``ctas`` contiguous ranges of
-// equal size, one per persistent CTA. A (sequence, kv head) segment cut by a
-// range boundary yields one partial per CTA that holds part of it, in slot
-// segment + CTA (unique: walking the pieces in order, segment + CTA grows by
-// one or two at each step).
+// The CTAs form groups of H_kv, one CTA per kv head; CTA c serves kv head
+// c % H_kv. The U = sum_b ceil(len_b / 128) units (sequence b, 128-key tile)
+// are cut into one contiguous range of equal size per group, so the H_kv
+// CTAs of a group read the same token rows of the cache (every head of a
+// token lies in one row) at about the same time. A (sequence, kv head)
+// segment cut by a range boundary yields one partial per group holding part
+// of it, in slot (b + group) * H_kv + kv head (unique: along one head's walk
+// b + group grows by one or two at each piece).
 struct DecodeTArgs {
-  int ctas;          // persistent CTAs (one per SM)
-  int* seg_first;    // [B * H_kv] first CTA holding a tile of the segment
-  int* seg_last;     // [B * H_kv] last such CTA
+  int ctas;          // persistent CTAs: groups * H_kv
+  int* seg_first;    // [B * H_kv] first group holding a tile of the segment
+  int* seg_last;     // [B * H_kv] last such group
   float* o_part;     // [(B * H_kv + ctas) * n_rows, D] fp32 partial O / l
   float* lse_part;   // [(B * H_kv + ctas) * n_rows] fp32 partial LSE
 };
@@ -25,9 +27,10 @@ struct DecodeTArgs {
 // Host: whether the balanced kernel takes a decode of this shape.
 inline bool decode_t_eligible(int D, long long n_rows) { return D == 128 && n_rows <= 64; }
 
-// Host: persistent CTAs on the current device (its SM count; 148 when the
-// device cannot be queried).
-int decode_t_ctas();
+// Host: persistent CTAs on the current device for H_kv kv heads: the most
+// whole groups of H_kv that fit its SM count (148 when the device cannot be
+// queried), at least one group.
+int decode_t_ctas(int H_kv);
 
 // Host: workspace bytes for the balanced decode: o_part, lse_part, seg_first
 // and seg_last, each rounded up to 256 bytes.

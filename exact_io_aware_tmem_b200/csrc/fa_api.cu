@@ -255,7 +255,7 @@ size_t fa_decode_workspace_size(int B, int q_len, int H, int H_kv, int D, int ma
   if (n_split == 0 && H % H_kv == 0 &&
       fa::decode_t_eligible(D, static_cast<long long>(q_len) * (H / H_kv)))
     return fa::decode_t_workspace(B, H_kv, static_cast<long long>(q_len) * (H / H_kv),
-                                  fa::decode_t_ctas());
+                                  fa::decode_t_ctas(H_kv));
   const int ns = fa_decode_num_splits(B, H_kv, max_seqlen_k, n_split);
   if (ns <= 1) return 0;
   const size_t rows = static_cast<size_t>(ns) * B * q_len * H;
@@ -344,7 +344,7 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, voi
     // Balanced partition over one persistent CTA per SM (decode_t.cu); the
     // workspace size above was computed for the same device.
     fa::DecodeTArgs t = {};
-    t.ctas = fa::decode_t_ctas();
+    t.ctas = fa::decode_t_ctas(H_kv);
     fa::decode_t_carve(t, workspace, B, H_kv, d.n_rows);
     return fa::cuda_status(fa::launch_decode_t(p, d, t, s));
   }

@@ -106,7 +106,8 @@ DEC_SPANS = [
 
 
 def spans(stamps, kinds: dict, table, n_steps: int, skip: int = 2) -> list:
-    """(label, median cycles, count) for each span of ``table``."""
+    """(label, median, mean, 90th percentile cycles, count) for each span of
+    ``table``."""
     out = []
     for label, a, da, b, db in table:
         d = []
@@ -117,7 +118,12 @@ def spans(stamps, kinds: dict, table, n_steps: int, skip: int = 2) -> list:
             x, y = int(stamps[kinds[a]][ta]), int(stamps[kinds[b]][tb])
             if x and y:
                 d.append(y - x)
-        out.append((label, statistics.median(d) if d else None, len(d)))
+        if d:
+            d.sort()
+            out.append((label, statistics.median(d), statistics.fmean(d),
+                        d[min(len(d) - 1, int(0.9 * len(d)))], len(d)))
+        else:
+            out.append((label, None, None, None, 0))
     return out
 
 
@@ -222,10 +228,18 @@ def main(argv=None) -> int:
     stamps, n = run(args.kernel, args.workload, args.cta)
     kinds, table = {"bwd": (BWD_KINDS, BWD_SPANS), "fwd": (FWD_KINDS, FWD_SPANS),
                     "dec": (DEC_KINDS, DEC_SPANS)}[args.kernel]
-    print(f"{args.kernel} {args.workload} CTA {args.cta}: {n} steps stamped; median cycles "
-          f"over the steady-state steps")
-    for label, med, cnt in spans(stamps, kinds, table, n):
-        print(f"  {label:62s} {'-' if med is None else f'{med:8.0f}'}  ({cnt})")
+    print(f"{args.kernel} {args.workload} CTA {args.cta}: {n} steps stamped; cycles over "
+          f"the steady-state steps")
+    nz = stamps[stamps != 0]
+    if nz.size:
+        span = int(nz.max()) - int(nz.min())
+        print(f"  first to last stamp: {span} cycles, {span / max(n, 1):.0f} per step")
+    print(f"  {'':62s} {'median':>8s} {'mean':>8s} {'p90':>8s}")
+    for label, med, mean, p90, cnt in spans(stamps, kinds, table, n):
+        if med is None:
+            print(f"  {label:62s} {'-':>8s}  (0)")
+        else:
+            print(f"  {label:62s} {med:8.0f} {mean:8.0f} {p90:8.0f}  ({cnt})")
     return 0
 
 

@@ -188,12 +188,13 @@ def test_decode_split_count_and_workspace_size(lib):
 def test_balanced_decode_workspace_size(lib):
     # Automatic splits at D = 128 with q_len * g <= 64 take the balanced
     # kernel: partial rows for (B * H_kv + CTAs) slots, plus two int arrays
-    # of B * H_kv. Without a device the library assumes 148 CTAs (B200 SMs).
+    # of B * H_kv. The CTAs are whole groups of H_kv; without a device the
+    # library assumes 148 SMs (B200).
     def r256(x):
         return (x + 255) // 256 * 256
-    for B, q_len, H, H_kv in [(16, 1, 32, 8), (16, 8, 32, 8), (3, 16, 16, 4)]:
+    for B, q_len, H, H_kv in [(16, 1, 32, 8), (16, 8, 32, 8), (3, 16, 16, 4), (2, 1, 5, 5)]:
         segs = B * H_kv
-        rows = (segs + 148) * q_len * (H // H_kv)
+        rows = (segs + 148 // H_kv * H_kv) * q_len * (H // H_kv)
         want = r256(rows * 128 * 4) + r256(rows * 4) + 2 * r256(segs * 4)
         assert lib.fa_decode_workspace_size(B, q_len, H, H_kv, 128, 32768, 0) == want
     # more than 64 rows (16 tokens x 8 heads), or an explicit split count:

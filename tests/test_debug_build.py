@@ -86,5 +86,23 @@ def test_debug_build_stamps_form_a_timeline(debug_lib, kernel):
     s = stamps[kinds[first]][:n].astype(np.int64)
     assert (np.diff(s) > 0).all()
     table = trace.BWD_SPANS if kernel == "bwd" else trace.FWD_SPANS
-    for label, med, cnt in trace.spans(stamps, kinds, table, n):
+    for label, med, mean, p90, cnt in trace.spans(stamps, kinds, table, n):
+        assert med is not None and cnt > 0 and med <= p90, label
+
+
+@pytest.mark.gpu
+def test_debug_build_decode_stamps(debug_lib):
+    """One traced CTA of the balanced decode (16 sequences, 64-row pages):
+    its group of H_kv CTAs takes an equal share of the (sequence, key tile)
+    units, and the CTA publishes each of its tiles in order."""
+    from exact_io_aware_tmem_b200.workloads import DECODE_WORKLOADS
+    name = "bf16_decode_paged64_b16_h32_kv8_d128_q1"
+    w = DECODE_WORKLOADS[name]
+    units = sum(-(-n // 128) for n in w.lengths())
+    groups = 148 // w.H_kv
+    stamps, n = trace.run("dec", name, cta=5)
+    assert n in (units // groups, units // groups + 1)
+    s = stamps[trace.DEC_KINDS["W_ARR"]][:n].astype(np.int64)
+    assert (np.diff(s) > 0).all()
+    for label, med, mean, p90, cnt in trace.spans(stamps, trace.DEC_KINDS, trace.DEC_SPANS, n):
         assert med is not None and cnt > 0, label
