@@ -110,8 +110,30 @@ struct Bars {
   }
 };
 
-// Event kinds of the debug build's stamps (index: the CTA's tile counter).
-enum : int { T_P_K = 0, T_P_V = 1, T_M_S = 2, T_M_PV = 3, T_W_SFULL = 4, T_W_ARR = 5, T_W_EPI = 6 };
+// Event kinds of the debug build's stamps (index: the CTA's tile counter),
+// and of its per-CTA records (index: the CTA): the SM it ran on, and the
+// global timer (ns) at its start and end.
+enum : int {
+  T_P_K = 0, T_P_V = 1, T_M_S = 2, T_M_PV = 3, T_W_SFULL = 4, T_W_ARR = 5, T_W_EPI = 6,
+  T_CTA_SM = 29, T_CTA_START = 30, T_CTA_END = 31
+};
+
+// Debug builds only: every CTA (below 1024) records its SM and the global
+// timer at its start and end into the trace buffer, whichever CTA is traced.
+__device__ __forceinline__ void cta_span(const AttnParams& p, int kind) {
+#ifdef FA_DEBUG
+  if (p.trace != nullptr && blockIdx.x < 1024) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    p.trace[kind * 1024 + blockIdx.x] = t;
+    if (kind == T_CTA_START) {
+      unsigned sm;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+      p.trace[T_CTA_SM * 1024 + blockIdx.x] = sm + 1ull;
+    }
+  }
+#endif
+}
 
 // Codes recorded in the device error word.
 enum : unsigned {
@@ -308,6 +330,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int R = dec.n_rows;
 
   if (threadIdx.x == 0) {
+    cta_span(p, T_CTA_START);
     *abort = 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bars.k_full(s), 1);
@@ -946,6 +969,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  if (threadIdx.x == 0) cta_span(p, T_CTA_END);
 }
 
 // Merge of the partials of one output row per warp: LSE = ln sum_c exp(LSE_c),

@@ -21,6 +21,8 @@ import argparse
 import statistics
 import sys
 
+import numpy as np
+
 # Event kinds, as numbered in the kernels' sources.
 BWD_KINDS = {
     "P_Q": 0, "P_DO": 1, "M_PREADY": 2, "M_SNEXT": 3, "M_DSREADY": 4, "M_DQ": 5,
@@ -90,6 +92,10 @@ FWD_SPANS = [
     ("producer: V_j issued before the MMA saw it", "P_V", 0, "M_VFULL", 0),
 ]
 
+
+# Per-CTA records of the balanced decode (index = CTA): SM + 1, and the
+# global timer (ns) at the CTA's start and end.
+DEC_CTA_SM, DEC_CTA_START, DEC_CTA_END = 29, 30, 31
 
 DEC_SPANS = [
     ("producer: K_j issued -> S_j issued (K landed, S buffer free)", "P_K", 0, "M_S", 0),
@@ -230,6 +236,17 @@ def main(argv=None) -> int:
                     "dec": (DEC_KINDS, DEC_SPANS)}[args.kernel]
     print(f"{args.kernel} {args.workload} CTA {args.cta}: {n} steps stamped; cycles over "
           f"the steady-state steps")
+    if args.kernel == "dec":
+        st, en = stamps[DEC_CTA_START].astype(np.int64), stamps[DEC_CTA_END].astype(np.int64)
+        ok = (st != 0) & (en != 0)
+        if ok.any():
+            t0 = st[ok].min()
+            dur = (en[ok] - st[ok]) / 1e3
+            print(f"  CTAs: {int(ok.sum())}, all done {(en[ok].max() - t0) / 1e3:.1f} us after the "
+                  f"first started; start spread {(st[ok].max() - t0) / 1e3:.1f} us; duration "
+                  f"min {dur.min():.1f} median {np.median(dur):.1f} max {dur.max():.1f} us")
+        stamps = stamps.copy()
+        stamps[DEC_CTA_SM:DEC_CTA_END + 1] = 0
     nz = stamps[stamps != 0]
     if nz.size:
         span = int(nz.max()) - int(nz.min())

@@ -104,5 +104,9 @@ def test_debug_build_decode_stamps(debug_lib):
     assert n in (units // groups, units // groups + 1)
     s = stamps[trace.DEC_KINDS["W_ARR"]][:n].astype(np.int64)
     assert (np.diff(s) > 0).all()
+    # every CTA's SM and span
+    sm, st, en = (stamps[k][:groups * w.H_kv].astype(np.int64)
+                  for k in (trace.DEC_CTA_SM, trace.DEC_CTA_START, trace.DEC_CTA_END))
+    assert (sm >= 1).all() and (sm <= 148).all() and (en > st).all() and (st > 0).all()
     for label, med, mean, p90, cnt in trace.spans(stamps, trace.DEC_KINDS, trace.DEC_SPANS, n):
         assert med is not None and cnt > 0, label
