@@ -124,6 +124,7 @@ def source_sha(*names) -> str:
 
 KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
                   "fwd_pair_kernel": ("fwd_pair.cu", "common.cuh", "params.h"),
+                  "fwd_d64_kernel": ("fwd_d64.cu", "fwd_d64.h", "common.cuh", "params.h"),
                   "bwd_fused_kernel": ("bwd_fused.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
@@ -394,7 +395,7 @@ def run_ours(args, w) -> None:
     do_bwd = w.backward
     ins = (q, k, v, do) if do_bwd else (q, k, v)
     bytes_in = sum(t.numel() * t.element_size() for t in ins)
-    fwd_name = "fwd_pair_kernel" if w.D == 128 else "fwd_bf16_kernel"
+    fwd_name = "fwd_pair_kernel" if w.D == 128 else "fwd_d64_kernel"
 
     def step(ev=None):
         if ev is not None:

@@ -9,6 +9,7 @@
 
 #include "../../include/fa.h"
 #include "decode_t.h"
+#include "fwd_d64.h"
 #include "params.h"
 
 namespace fa {
@@ -232,7 +233,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.err.word = fa::err_word();
   if (p.err.word == nullptr) return FA_ERR_CUDA;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e = (dtype == FA_F32) ? fa::launch_fwd_f32(p, s) : fa::launch_fwd_bf16(p, s);
+  const cudaError_t e = (dtype == FA_F32) ? fa::launch_fwd_f32(p, s)
+                        : (D == 64)       ? fa::launch_fwd_d64(p, s)
+                                          : fa::launch_fwd_bf16(p, s);
   return fa::cuda_status(e);
 }
 
