@@ -388,8 +388,16 @@ def run_ours(args, w) -> None:
     lse = torch.empty((B, w.H, w.N) if not inp.varlen else (w.H, T), device=dev,
                       dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(fa.workspace_size(T, w.H, w.D, q.dtype), dtype=torch.uint8, device=dev)
-    ph = fa.BWD_FUSED  # preprocess (+ accumulator zeroing), fused kernel, dQ conversion
+    ws = torch.empty(max(fa.workspace_size(T, w.H, w.D, q.dtype),
+                         fa.workspace_size(T, w.H, w.D, q.dtype, fa.BWD_SPLIT)),
+                     dtype=torch.uint8, device=dev)
+    # The backward's three kernels: preprocess (+ accumulator zeroing), fused
+    # kernel, dQ conversion; or, with --bwd split, preprocess, dK / dV kernel,
+    # dQ kernel (the reproducible split backward).
+    split = getattr(args, "bwd", "fused") == "split"
+    ph_steps = (0x01, 0x02, 0x04) if split else (0x01, 0x08, 0x10)
+    bwd_names = (("bwd_preprocess", "bwd_dkdv_kernel", "bwd_dq_kernel") if split else
+                 ("bwd_preprocess", "bwd_fused_kernel", "dq_convert"))
     # Forward-only workloads (the B4 N2048 D64 configuration) time the
     # forward alone: their step is one fa_fwd.
     do_bwd = w.backward
@@ -405,15 +413,10 @@ def run_ours(args, w) -> None:
             ev[1].record()
         if not do_bwd:
             return
-        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph & 0x01, **kw)
-        if ev is not None:
-            ev[2].record()
-        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph & 0x08, **kw)
-        if ev is not None:
-            ev[3].record()
-        fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph & 0x10, **kw)
-        if ev is not None:
-            ev[4].record()
+        for i, ph in enumerate(ph_steps):
+            fa.bwd(do, q, k, v, o, lse, workspace=ws, dq=dq, dk=dk, dv=dv, phases=ph, **kw)
+            if ev is not None:
+                ev[2 + i].record()
 
     for _ in range(args.warmup):
         step()
@@ -450,7 +453,7 @@ def run_ours(args, w) -> None:
     max_ms = reduce_max(elapsed_ms, dev)
     spans = {fwd_name: (0, 1)}
     if do_bwd:
-        spans.update({"bwd_preprocess": (1, 2), "bwd_fused_kernel": (2, 3), "dq_convert": (3, 4)})
+        spans.update({name: (1 + i, 2 + i) for i, name in enumerate(bwd_names)})
     k_ms = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
             for name, (a, b) in spans.items()}
     k_ms = {n: reduce_max(t, dev) for n, t in k_ms.items()}
@@ -468,7 +471,7 @@ def run_ours(args, w) -> None:
         if do_bwd:
             gq, gk, gv = outs_[2:]
             fa.bwd(ins_[3], qq, kk, vv, outs_[0], outs_[1], workspace=ws, dq=gq, dk=gk, dv=gv,
-                   **kw)
+                   phases=fa.BWD_SPLIT if split else fa.BWD_FUSED, **kw)
 
     if world > 1:
         dist.barrier()
@@ -488,14 +491,17 @@ def run_ours(args, w) -> None:
     fwd_tf = fwd_fl / (k_ms[fwd_name] / 1e3) / 1e12
     bwd_tf = None
     if do_bwd:
-        bwd_ms = k_ms["bwd_preprocess"] + k_ms["bwd_fused_kernel"] + k_ms["dq_convert"]
+        bwd_ms = sum(k_ms[n] for n in bwd_names)
         bwd_tf = bwd_fl / (bwd_ms / 1e3) / 1e12
-    # Dominant kernel: the one with the largest share of the step. Algorithmic
-    # FLOPs per launch: the forward's two products (4 N^2 D per head) and the
-    # fused backward's five (S, dP, dV, dK, dQ: 10 N^2 D, the method's 2.5x),
-    # causal halving each.
+    # Dominant kernel: the one with the largest share of the step. FLOPs per
+    # launch: the forward's two products (4 N^2 D per head) and the fused
+    # backward's five (S, dP, dV, dK, dQ: 10 N^2 D, the method's 2.5x), causal
+    # halving each; the split backward's kernels count the products they run
+    # (dK / dV kernel: S, dP, dV, dK; dQ kernel: S, dP, dQ).
     kernel_fl = {fwd_name: fwd_fl}
-    if do_bwd:
+    if do_bwd and split:
+        kernel_fl.update({"bwd_dkdv_kernel": 2.0 * fwd_fl, "bwd_dq_kernel": 1.5 * fwd_fl})
+    elif do_bwd:
         kernel_fl["bwd_fused_kernel"] = bwd_fl
     dom = max(kernel_fl, key=lambda n: k_ms[n])
     dom_fl = kernel_fl[dom]
@@ -506,6 +512,8 @@ def run_ours(args, w) -> None:
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(config_of(w), parallelism=f"replicas{world}" if world > 1 else "none",
+                       backward=("split (dK / dV kernel + dQ kernel)" if split else "fused")
+                       if do_bwd else None,
                        l2=f"not flushed: every step reads and writes "
                           f"{(bytes_in + bytes_out) / 2**20:.0f} MiB > {L2_BYTES >> 20} MiB L2",
                        ranks="each rank its own seeded batch of this shape"),
@@ -950,6 +958,8 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bwd", choices=["fused", "split"], default="fused",
+                    help="backward path of the attention step (default: the fused kernel)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
     from exact_io_aware_tmem_b200.workloads import DECODE_WORKLOADS, WORKLOADS
