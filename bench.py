@@ -123,14 +123,14 @@ def source_sha(*names) -> str:
 
 
 KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
-                  "fwd_pair_kernel": ("fwd_pair.cu", "common.cuh", "params.h"),
+                  "fwd_pair_kernel": ("fwd_pair.cu", "fwd_fp8.h", "common.cuh", "params.h"),
                   "fwd_d64_kernel": ("fwd_d64.cu", "fwd_d64.h", "common.cuh", "params.h"),
                   "bwd_fused_kernel": ("bwd_fused.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "decode": ("fwd_bf16.cu", "common.cuh", "params.h"),
                   "decode_t": ("decode_t.cu", "decode_t.h", "common.cuh", "params.h"),
-                  "fp8_fwd": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "fp8_fwd": ("fwd_pair.cu", "fwd_fp8.h", "common.cuh", "params.h"),
                   "fp8_quantize_kernel": ("fp8.cu", "common.cuh", "params.h")}
 
 
@@ -709,8 +709,8 @@ def run_fp8(args, name, w) -> None:
                        l2="not flushed: every step reads and writes > 200 MiB > 126 MiB L2",
                        ranks="each rank its own seeded batch of this shape"),
         "kernel_ms": {"fp8_quantize_kernel (Q and K)": round(q_ms, 4),
-                      "fwd_bf16_kernel<128, false, true>": round(f_ms, 4)},
-        "roofline": {"kernel": "fwd_bf16_kernel<128, false, true>", "bound": "tensor",
+                      "fwd_pair_kernel<128, e4m3>": round(f_ms, 4)},
+        "roofline": {"kernel": "fwd_pair_kernel<128, e4m3>", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
                      "peak_kind": f"{peaks['source']} {peak_kind} bf16 / 0.75 (E4M3 Q K^T at the "

@@ -10,6 +10,7 @@
 #include "../../include/fa.h"
 #include "decode_t.h"
 #include "fwd_d64.h"
+#include "fwd_fp8.h"
 #include "params.h"
 
 namespace fa {
@@ -387,7 +388,7 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v, const float*
   if (p.err.word == nullptr) return FA_ERR_CUDA;
   fa::Fp8Args f = {q_scale, k_scale, (N + 127) / 128};
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return fa::cuda_status(fa::launch_fwd_fp8(p, f, s));
+  return fa::cuda_status(fa::launch_fwd_pair_fp8(p, f, s));
 }
 
 size_t fa_bwd_phases_workspace_size(unsigned mask, long long total_tokens, int H, int D,

@@ -31,9 +31,16 @@
 // j+1 completing implies P_g V_j has completed (the tensor core runs one
 // thread's MMAs in order and a commit covers all earlier ones), so a group
 // can rescale its O between the two without any other signal.
+// F8 (D = 128): pass 2 of the FP8 forward (aiqz.cc article, section "FP8 low
+// precision"). Q and K arrive as E4M3 codes, one 128-byte row per token, with
+// one fp32 step per 128-token block (pass 1, fp8.cu); S = Q_hat K_hat^T runs
+// as a kind::f8f6f4 MMA with fp32 accumulation and is scaled by the two
+// blocks' Delta_Q Delta_K with the logit scale. P V stays bf16. The smaller Q
+// and K tiles leave room for four K and four V stages.
 #include <limits.h>
 #include <math.h>
 
+#include "fwd_fp8.h"
 #include "params.h"
 
 namespace fa {
@@ -53,15 +60,18 @@ constexpr uint32_t SPAN = 128 * 128;          // 128 rows x 128 bytes (one swizz
 constexpr int KS_MAX = 4;
 constexpr int VS_MAX = 4;
 
-template <int D>
+template <int D, bool F8>
 struct Cfg {
   static_assert(D == 64 || D == 128, "head dim");
-  static constexpr uint32_t TILE = BM * D * 2;       // 32 KB at D = 128
-  static constexpr int KS = D == 128 ? 3 : 4;        // K stages
-  static constexpr int VS = D == 128 ? 2 : 4;        // V stages
+  static_assert(!F8 || D == 128, "E4M3 rows of 128 bytes");
+  static constexpr uint32_t TILE = BM * D * 2;       // bf16 tile, 32 KB at D = 128
+  static constexpr uint32_t QK_TILE = F8 ? BM * D : TILE;   // Q or K tile
+  static constexpr int QK_CHUNKS = F8 ? 1 : D / 64;  // 128-byte column blocks of a Q / K row
+  static constexpr int KS = F8 ? 4 : (D == 128 ? 3 : 4);   // K stages
+  static constexpr int VS = F8 ? 4 : (D == 128 ? 2 : 4);   // V stages
   static constexpr uint32_t OFF_Q = 0;               // Q_0, Q_1
-  static constexpr uint32_t OFF_K = OFF_Q + 2 * TILE;
-  static constexpr uint32_t OFF_V = OFF_K + KS * TILE;
+  static constexpr uint32_t OFF_K = OFF_Q + 2 * QK_TILE;
+  static constexpr uint32_t OFF_V = OFF_K + KS * QK_TILE;
   static constexpr uint32_t OFF_BAR = OFF_V + VS * TILE;
   // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2],
   // p_ready[2], o_full (laid out for the largest ring depths)
@@ -109,15 +119,16 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
 
 // 320 threads: ten warps, three on two of the four SM sub-partitions, whose
 // 16K registers then allow 168 per thread.
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m2,
-                    int group) {
-  using C = Cfg<D>;
+                    int group, const Fp8Args f8) {
+  using C = Cfg<D, F8>;
   constexpr int KS = C::KS, VS = C::VS;
-  constexpr uint32_t TILE = C::TILE, OFF_Q = C::OFF_Q, OFF_K = C::OFF_K, OFF_V = C::OFF_V;
+  constexpr uint32_t TILE = C::TILE, QK_TILE = C::QK_TILE;
+  constexpr uint32_t OFF_Q = C::OFF_Q, OFF_K = C::OFF_K, OFF_V = C::OFF_V;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if ((sbase & 1023u) != 0) {
@@ -185,11 +196,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&tm_v);
       // Both query tiles; rows past the tensor arrive as zeros (and are
       // never written out).
-      mbar_arrive_expect_tx(bars.q_full(), 2 * TILE);
+      mbar_arrive_expect_tx(bars.q_full(), 2 * QK_TILE);
       for (int g = 0; g < 2; ++g)
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sbase + OFF_Q + g * TILE + c * SPAN, &tm_q, bars.q_full(), h * D + c * 64,
-                      sq.start + (2 * m2 + g) * BM);
+        for (int c = 0; c < C::QK_CHUNKS; ++c)
+          tma_load_2d(sbase + OFF_Q + g * QK_TILE + c * SPAN, &tm_q, bars.q_full(),
+                      h * D + c * 64, sq.start + (2 * m2 + g) * BM);
     }
     int jk = 0, jv = 0;
     long long t_last = clock64();
@@ -199,9 +210,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           __all_sync(FULL, mbar_try_wait(bars.k_empty(jk % KS), ((jk / KS) & 1) ^ 1))) {
         const int st = jk % KS;
         if (lane == 0) {
-          mbar_arrive_expect_tx(bars.k_full(st), TILE);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sbase + OFF_K + st * TILE + c * SPAN, &tm_k, bars.k_full(st),
+          mbar_arrive_expect_tx(bars.k_full(st), QK_TILE);
+          for (int c = 0; c < C::QK_CHUNKS; ++c)
+            tma_load_2d(sbase + OFF_K + st * QK_TILE + c * SPAN, &tm_k, bars.k_full(st),
                         hk * D + c * 64, sq.start + jk * BN);
           FA_STAMP(p, T_P_K, jk);
         }
@@ -254,18 +265,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     // one elected lane issues the tensor-core instructions and commits.
     const uint32_t leader = elect_one();
     constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
+    constexpr uint32_t IDESC_QK8 = idesc_e4m3(BM, BN);
     constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
     const uint64_t q_desc = sdesc_sw128(sbase + OFF_Q, 16, 1024);
     const uint64_t k_desc = sdesc_sw128(sbase + OFF_K, 16, 1024);
     const uint64_t v_desc = sdesc_sw128(sbase + OFF_V, SPAN, 1024);
-    // S_g = Q_g K_j^T (M = 128 rows, N = 128 keys, K = D in steps of 16).
+    // S_g = Q_g K_j^T (M = 128 rows, N = 128 keys, K = D in steps of 16
+    // bf16 or 32 E4M3 codes: 32 bytes of a row either way).
     auto issue_s = [&](int g, int j) {
       const int st = j % KS;
+      if constexpr (F8) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t o = (kk >> 2) * SPAN + (kk & 3) * 32;
-        mma_ss_if(leader, tmem + TM_S + g * BN, sdesc_add(q_desc, g * TILE + o),
-                  sdesc_add(k_desc, st * TILE + o), IDESC_QK, kk > 0);
+        for (int kk = 0; kk < D / 32; ++kk)
+          mma_ss_e4m3_if(leader, tmem + TM_S + g * BN, sdesc_add(q_desc, g * QK_TILE + kk * 32),
+                         sdesc_add(k_desc, st * QK_TILE + kk * 32), IDESC_QK8, kk > 0);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * SPAN + (kk & 3) * 32;
+          mma_ss_if(leader, tmem + TM_S + g * BN, sdesc_add(q_desc, g * TILE + o),
+                    sdesc_add(k_desc, st * TILE + o), IDESC_QK, kk > 0);
+        }
       }
       tc_commit_if(leader, bars.s_full(g));
     };
@@ -330,14 +350,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_col = tmem + lane_off + TM_S + g * BN;
     const uint32_t o_col = tmem + lane_off + TM_O + g * D;
-    const float c2 = p.scale_log2;
     const int n = g ? n_1 : n_0;
+    // Logit scale in log2 units per raw score; E4M3 scores are in units of
+    // Delta_Q Delta_K of their two blocks (Delta_K per key tile below).
+    float c2 = p.scale_log2;
+    const float* kscale_row = nullptr;
+    if constexpr (F8) {
+      if (n > 0) c2 *= __ldg(f8.q_scale + (static_cast<size_t>(b) * p.H + h) * f8.n_blocks +
+                             2 * m2 + g);
+      kscale_row = f8.k_scale + (static_cast<size_t>(b) * p.H_kv + hk) * f8.n_blocks;
+    }
     const bool stamp = quarter == 0 && lane == 0;   // debug stamps: first warp of each group
     [[maybe_unused]] const int tk = 4 * g;
     float m_ref = -INFINITY;  // reference max (log2 units)
     float l = 0.f;            // row sum in that reference
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
+      const float c2t = F8 ? c2 * __ldg(kscale_row + j) : c2;   // log2 units per raw score
       if (!(ok = warp_wait(bars.s_full(g), j & 1, p.err, abort, W_SFULL))) break;
       if (stamp) FA_STAMP(p, T_W_SFULL + tk, j);
       tc_fence_after();
@@ -365,7 +394,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(r[c][i]));
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      const float m_cand = mx * c2;
+      const float m_cand = mx * c2t;
       const bool grow = m_cand > m_ref + RESCALE_LOG2;   // always true on the first visible tile
       const float m_new = grow ? m_cand : m_ref;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
@@ -375,8 +404,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use));
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2t, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2t, -m_use));
           sum4[(i >> 1) & 3] += p0 + p1;
           pk[i >> 1] = pack_bf16x2(p0, p1);
         }
@@ -457,7 +486,7 @@ namespace {
 template <int D>
 cudaError_t launch_pair_d(const AttnParams& p, cudaStream_t stream) {
   using namespace pair;
-  using C = Cfg<D>;
+  using C = Cfg<D, false>;
   const int num_m2 = (p.max_seqlen + 2 * BM - 1) / (2 * BM);
   const long long tiles = static_cast<long long>(num_m2) * p.H * p.B;
   if (tiles == 0 || p.total == 0) return cudaSuccess;
@@ -467,16 +496,41 @@ cudaError_t launch_pair_d(const AttnParams& p, cudaStream_t stream) {
       !make_tmap_bf16_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN) ||
       !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_pair_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_pair_kernel<D, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int group = l2_group(4ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_pair_kernel<D><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(tq, tk, tv, p,
-                                                                                 num_m2, group);
+  fwd_pair_kernel<D, false><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, num_m2, group, Fp8Args{});
   return cudaGetLastError();
 }
 
 }  // namespace
+
+// Pass 2 of the FP8 forward at D = 128: p.q / p.k hold the E4M3 codes, ``f``
+// their per-block steps (fa_fwd_fp8 uses it).
+cudaError_t launch_fwd_pair_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream) {
+  using namespace pair;
+  constexpr int D = 128;
+  using C = Cfg<D, true>;
+  if (p.D != D) return cudaErrorInvalidValue;
+  const int num_m2 = (p.max_seqlen + 2 * BM - 1) / (2 * BM);
+  const long long tiles = static_cast<long long>(num_m2) * p.H * p.B;
+  if (tiles == 0 || p.total == 0) return cudaSuccess;
+  if (tiles > INT_MAX) return cudaErrorInvalidConfiguration;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_u8_2d(&tq, p.q, p.total, static_cast<unsigned long long>(p.H) * D, 128, BM) ||
+      !make_tmap_u8_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 128, BN) ||
+      !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_pair_kernel<D, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int group = l2_group(3ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
+  fwd_pair_kernel<D, true><<<static_cast<unsigned>(tiles), THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, num_m2, group, f);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fwd_pair(const AttnParams& p, cudaStream_t stream) {
   if (p.D == 64) return launch_pair_d<64>(p, stream);
