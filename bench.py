@@ -122,15 +122,14 @@ def source_sha(*names) -> str:
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "params.h"),
-                  "fwd_pair_kernel": ("fwd_pair.cu", "fwd_fp8.h", "common.cuh", "params.h"),
+KERNEL_SOURCES = {"fwd_pair_kernel": ("fwd_pair.cu", "common.cuh", "params.h"),
                   "fwd_d64_kernel": ("fwd_d64.cu", "fwd_d64.h", "common.cuh", "params.h"),
                   "bwd_fused_kernel": ("bwd_fused.cu", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
-                  "decode": ("fwd_bf16.cu", "common.cuh", "params.h"),
+                  "decode": ("decode_split.cu", "common.cuh", "params.h"),
                   "decode_t": ("decode_t.cu", "decode_t.h", "common.cuh", "params.h"),
-                  "fp8_fwd": ("fwd_pair.cu", "fwd_fp8.h", "common.cuh", "params.h"),
+                  "fp8_fwd": ("fwd_pair.cu", "common.cuh", "params.h"),
                   "fp8_quantize_kernel": ("fp8.cu", "common.cuh", "params.h")}
 
 
@@ -932,7 +931,7 @@ def run_decode(args, w) -> None:
         "tflops": fl / (call_ms / 1e3) / 1e12,
         "kernel_ms": {"fa_decode (partials + merge)": round(call_ms, 4)},
         "roofline": {"kernel": ("decode_t_kernel + decode_t_merge_kernel" if balanced else
-                                "fwd_bf16_kernel<decode> + decode_combine_kernel") +
+                                "decode_split_kernel + decode_combine_kernel") +
                                " (one fa_decode)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peaks['source']} HBM copy",

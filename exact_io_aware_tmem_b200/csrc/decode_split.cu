@@ -1,30 +1,31 @@
-// Attention forward, bf16 in / fp32 accumulate, on the sm_100a tensor cores.
+// Split-KV decode over a contiguous or paged bf16 KV cache, on the sm_100a
+// tensor cores: the form fa_decode takes when the caller fixes the number of
+// key splits, or when the balanced kernel (decode_t.cu) does not take the
+// shape (D = 64, or more than 64 query rows per kv head).
 //
-// What it computes: for every query row, the online-softmax recurrence of
+// What it computes: the q_len newest tokens of each sequence attend to its
+// cached keys (agentalpha.top "flash attention" answer, follow-up 2: the key
+// range is cut into splits, each split runs the online-softmax recurrence of
 // aiqz.cc "Flash Attention V2/V3 optimization", section "V2 algorithm
-// optimisation" (steps 1-5): over key tiles j,
+// optimisation" (steps 1-5) over its key tiles j,
 //     m_new = max(m, rowmax(S_j)),  alpha = e^(m - m_new),
 //     l = l * alpha + rowsum(e^(S_j - m_new)),
 //     O = O * alpha + e^(S_j - m_new) V_j,
-// then O / l once at the end, with S = scale * Q K^T (scale before the max,
-// as in the same article's Python demo) and LSE = m + ln l saved for the
-// backward pass (airsota.com card, section 4 item 2). Exponentials are taken
-// in base 2 on pre-scaled logits (scale * log2 e), which is the same
-// recurrence up to rounding.
+// and the splits' (O / l, LSE) pairs are merged with the same update). S =
+// scale * Q K^T, exponentials in base 2 on pre-scaled logits.
 //
-// How, on B200 (one CTA per 128-row Q tile; 352 threads at D = 128, 320 at
-// D = 64):
+// How, on B200 (one CTA per (sequence, kv head, split); 352 threads at
+// D = 128, 320 at D = 64). The CTA's 128 TMEM lanes hold the q_len x g query
+// rows of one kv head (row r = token r / g of head hk * g + r % g):
 //   warp 8      TMA producer (the whole warp runs its loop, lane 0 issues):
-//               the Q tile once, then K_j and V_j tiles through separate
+//               the Q block once, then K_j and V_j tiles through separate
 //               multi-stage shared-memory rings (mbarrier full/empty pairs,
 //               128-byte swizzle, no multicast), K loaded ahead of V whenever
-//               both rings have room;
+//               both rings have room; one box per page of a paged cache;
 //   warp 9      MMA warp, converged, one elect.sync lane issuing: S_j =
 //               Q K_j^T with tcgen05.mma into TMEM score buffer j mod 2 (Q is
-//               the A operand, held in TMEM, so each tile streams only K and
-//               V through shared memory and the tensor core is not held back
-//               by shared-memory bandwidth) as soon as the softmax has loaded
-//               S_{j-2};
+//               the A operand, held in TMEM) as soon as the softmax has
+//               loaded S_{j-2};
 //   warp 10     (D = 128) the same for O += P_j V_j, with P read straight
 //               from its own TMEM columns as packed bf16. At D = 64 warp 9
 //               issues these too, QK_{j+2} ahead of each PV_j;
@@ -35,12 +36,9 @@
 //               exponentiates, sums, stores P to TMEM and rescales its O row
 //               in TMEM when the reference max moved. Group 0 first copies Q
 //               from the swizzled shared tile into TMEM. At the end both
-//               groups merge their row sums and each writes half of O / l.
-// The same pipeline has two more instantiations (template flags, below):
-// split-KV decode over a contiguous or paged KV cache (agentalpha.top
-// "flash attention" answer, follow-up 2) and the FP8 (E4M3) forward, whose
-// score MMA reads E4M3 Q and K from shared memory (aiqz.cc article, section
-// "FP8 low precision").
+//               groups merge their row sums and each writes half of O / l
+//               (fp32 partials for the merge kernel when there are several
+//               splits, else the final bf16 O and LSE).
 // The two groups run the same recurrence with one shared reference max per
 // row: the group on tile j takes the reference of tile j-1 from the other
 // group (a shared-memory word per row, published by an mbarrier arrive as
@@ -83,12 +81,9 @@ enum : unsigned {
   W_VTAIL = 0x10E00, BAD_CACHE_LEN = 0x10F01, BAD_PAGE = 0x10F02
 };
 
-// F8: Q and K are E4M3 tiles (one 128-byte row per token at D = 128) that
-// the score MMA reads from shared memory; V stays bf16.
-template <int D, bool F8>
-struct FwdCfg {
-  static_assert(!F8 || D == 128, "the E4M3 path has one 128-byte row per token");
-  static constexpr int STAGES = (D == 64 || F8) ? 4 : 3;
+template <int D>
+struct Cfg {
+  static constexpr int STAGES = (D == 64) ? 4 : 3;
   // D = 128: one warp issues the score MMAs and another the P V MMAs, so a
   // score MMA never waits behind the P V product of the tile before it.
   // D = 64 (half the MMA work per exponential): one warp issues both in a
@@ -96,19 +91,15 @@ struct FwdCfg {
   static constexpr bool SPLIT_MMA = D == 128;
   static constexpr int THREADS = SPLIT_MMA ? 352 : 320;
   static constexpr int CHUNKS = D / 64;            // 128-byte blocks of a bf16 row
-  static constexpr int QK_CHUNKS = F8 ? 1 : CHUNKS; // 128-byte blocks of a Q / K row
-  static_assert(QK_CHUNKS >= 1, "row blocks");
   static constexpr uint32_t TILE = BM * D * 2;     // bytes of one bf16 128-row tile
-  static constexpr uint32_t QK_TILE = F8 ? BM * D : TILE;
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + QK_TILE;
-  static constexpr uint32_t OFF_V = OFF_K + STAGES * QK_TILE;
+  static constexpr uint32_t OFF_K = OFF_Q + TILE;
+  static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
   // Per-row exchange words: reference max per group [2][128], then final
-  // (m, l) per group [2][2][128]. The bf16 paths keep them in the Q tile
-  // once Q is in TMEM; the E4M3 path reads Q from shared memory throughout.
+  // (m, l) per group [2][2][128], kept in the Q tile once Q is in TMEM.
   static constexpr uint32_t XCHG = 6 * BM * 4;
-  static constexpr uint32_t OFF_X = F8 ? OFF_V + STAGES * TILE : OFF_Q;
-  static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE + (F8 ? XCHG : 0);
+  static constexpr uint32_t OFF_X = OFF_Q;
+  static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
   // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
   // mref[2], pv_done[2], p_ready, q_tmem, fin, v_fix
   static constexpr int NBAR = 1 + 4 * STAGES + 12;
@@ -116,7 +107,7 @@ struct FwdCfg {
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr uint32_t OFF_MREF = OFF_X;
   static constexpr uint32_t OFF_FIN = OFF_X + 2 * BM * 4;
-  static_assert(F8 || XCHG <= QK_TILE, "exchange words fit in the Q tile");
+  static_assert(XCHG <= TILE, "exchange words fit in the Q tile");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -150,83 +141,58 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
   return __all_sync(FULL, ok);
 }
 
-// DEC = false: the forward over packed or dense sequences (one CTA per 128-row
-// Q tile). DEC = true: split-KV decode, one CTA per (sequence, kv head, key
-// split); its Q tile is the q_len newest tokens x the g query heads of the kv
-// head (rows r = token * g + head), and it writes that split's partial O / l
-// and LSE (or the final O and LSE when there is one split).
-// F8 = true: Q and K arrive as E4M3 codes with one fp32 step per 128-token
-// block (pass 1, fp8.cu); S = Q_hat K_hat^T runs as a kind::f8f6f4 MMA with
-// fp32 accumulation and is scaled by Delta_Q Delta_K of its two blocks.
-template <int D, bool DEC, bool F8>
-__global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
-    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
-                    const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p, int num_m,
-                    int group, const DecodeArgs dec, const Fp8Args f8) {
-  static_assert(!(DEC && F8), "the E4M3 path is a forward over dense batches");
-  using C = FwdCfg<D, F8>;
+// One CTA per (sequence, kv head, key split); its Q tile is the q_len newest
+// tokens x the g query heads of the kv head (rows r = token * g + head), and
+// it writes that split's partial O / l and LSE (or the final O and LSE when
+// there is one split).
+template <int D>
+__global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p,
+                        const DecodeArgs dec) {
+  using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
 
-  int m_blk = 0, h = 0, hk = 0, b = 0;
-  int j0 = 0;       // first key tile of this CTA
-  int n_kv = 0;     // key tiles of this CTA
-  int split = 0;
-  SeqInfo sq{0, 0}; // forward: the sequence; decode: start 0, len = keys in cache
-  if constexpr (!DEC) {
-    // Tile order: groups of heads for L2 reuse of K / V; inside a group the
-    // longest causal tiles (largest m_blk) first.
-    const TileSlot ts = grouped_slot(blockIdx.x, num_m, p.H * p.B, group);
-    m_blk = num_m - 1 - ts.t;
-    const int rem = ts.unit;
-    h = rem % p.H;
-    b = rem / p.H;
-    sq = seq_info(p, b);
-    if (!seq_ok(p, sq) || m_blk * BM >= sq.len) return;  // whole CTA, before any shared state
-    hk = h / (p.H / p.H_kv);
-    const int n_kv_all = (sq.len + BN - 1) / BN;
-    n_kv = p.causal ? min(n_kv_all, m_blk + 1) : n_kv_all;
-  } else {
-    split = blockIdx.x % dec.n_split;
-    const int rem = blockIdx.x / dec.n_split;
-    hk = rem % p.H_kv;
-    b = rem / p.H_kv;
-    sq.len = __ldg(dec.cache_seqlens + b);
-    if (sq.len < 0 || sq.len > p.max_seqlen) {
-      if (threadIdx.x == 0) record_bounds(p.err, BAD_CACHE_LEN);
-      return;
-    }
-    j0 = split * dec.chunk;
-    n_kv = min((sq.len + BN - 1) / BN - j0, dec.chunk);
-    if (n_kv <= 0) {
-      // No key in this split: LSE -inf and O 0, so the merge gives it no
-      // weight (the whole output when the sequence is empty).
-      const int r = threadIdx.x;
-      if (r < dec.n_rows) {
-        const int tok = b * dec.q_len + r / dec.g;
-        const int hq = hk * dec.g + r % dec.g;
-        const size_t row = static_cast<size_t>(tok) * p.H + hq;
-        if (dec.n_split == 1) {
-          p.lse[row] = -INFINITY;
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row * D);
-          for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-        } else {
-          const size_t prow = static_cast<size_t>(split) * p.total * p.H + row;
-          dec.lse_part[prow] = -INFINITY;
-          float4* dst = reinterpret_cast<float4*>(dec.o_part + prow * D);
-          for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      return;
-    }
+  const int split = blockIdx.x % dec.n_split;
+  const int rem = blockIdx.x / dec.n_split;
+  const int hk = rem % p.H_kv;
+  const int b = rem / p.H_kv;
+  const int len = __ldg(dec.cache_seqlens + b);   // keys in the cache
+  if (len < 0 || len > p.max_seqlen) {
+    if (threadIdx.x == 0) record_bounds(p.err, BAD_CACHE_LEN);
+    return;
   }
-  // Decode: the split holding the sequence's last, partly filled key tile
-  // zeroes that tile's V rows past the end (the cache may hold anything
-  // there, and 0 * NaN in P V would not be 0) before PV reads it.
-  const bool v_tail = DEC && j0 + n_kv == (sq.len + BN - 1) / BN && (sq.len % BN) != 0;
+  const int j0 = split * dec.chunk;                          // first key tile of this CTA
+  const int n_kv = min((len + BN - 1) / BN - j0, dec.chunk);  // key tiles of this CTA
+  if (n_kv <= 0) {
+    // No key in this split: LSE -inf and O 0, so the merge gives it no
+    // weight (the whole output when the sequence is empty).
+    const int r = threadIdx.x;
+    if (r < dec.n_rows) {
+      const int tok = b * dec.q_len + r / dec.g;
+      const int hq = hk * dec.g + r % dec.g;
+      const size_t row = static_cast<size_t>(tok) * p.H + hq;
+      if (dec.n_split == 1) {
+        p.lse[row] = -INFINITY;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row * D);
+        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+      } else {
+        const size_t prow = static_cast<size_t>(split) * p.total * p.H + row;
+        dec.lse_part[prow] = -INFINITY;
+        float4* dst = reinterpret_cast<float4*>(dec.o_part + prow * D);
+        for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    return;
+  }
+  // The split holding the sequence's last, partly filled key tile zeroes
+  // that tile's V rows past the end (the cache may hold anything there, and
+  // 0 * NaN in P V would not be 0) before PV reads it.
+  const bool v_tail = j0 + n_kv == (len + BN - 1) / BN && (len % BN) != 0;
 
   const Bars bars{sbase + C::OFF_BAR, C::STAGES};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -273,15 +239,11 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     // the next batch already in flight; a tile's ids then come by shuffle.
     // Looking each id up on its own put an L2 round trip in front of every
     // TMA issue. -1: a page past the sequence's end (or past the table row).
-    const int n_pages = DEC ? (sq.len + dec.page - 1) / max(dec.page, 1) : 0;
+    const int n_pages = (len + dec.page - 1) / max(dec.page, 1);
     auto page_id = [&](int pg) -> int {
-      if constexpr (DEC) {
-        return (pg < n_pages && pg < dec.max_blocks)
-                   ? __ldg(dec.block_table + static_cast<size_t>(b) * dec.max_blocks + pg)
-                   : -1;
-      } else {
-        return -1;
-      }
+      return (pg < n_pages && pg < dec.max_blocks)
+                 ? __ldg(dec.block_table + static_cast<size_t>(b) * dec.max_blocks + pg)
+                 : -1;
     };
     struct PageBatch {
       int base, cur, nxt;
@@ -305,26 +267,12 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       const int off = pg0 + min(lane, n - 1) - pb.base;   // < 32
       return __shfl_sync(FULL, pb.cur, off & 31);
     };
-    const bool paged = DEC && dec.block_table != nullptr;
+    const bool paged = dec.block_table != nullptr;
     const int box = paged ? min(dec.page, BN) : BN;   // rows per TMA box
     // K / V tile jt (absolute key tile) into shared memory at ``dst``. The
     // caller has posted the tile's expected bytes on ``bar``.
-    auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int jt, PageBatch& pb,
-                       bool is_k) {
-      if constexpr (F8) {
-        // E4M3 K: one 128-byte (128-code) column block; V: bf16 as below.
-        if (lane == 0) {
-          const int chunks = is_k ? 1 : C::CHUNKS;
-          for (int c = 0; c < chunks; ++c)
-            tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, sq.start + jt * BN);
-        }
-      } else if constexpr (!DEC) {
-        if (lane == 0) {
-#pragma unroll
-          for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_2d(dst + c * CHUNK_BYTES, map, bar, hk * D + c * 64, sq.start + jt * BN);
-        }
-      } else if (!paged) {
+    auto load_kv = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int jt, PageBatch& pb) {
+      if (!paged) {
         if (lane == 0) {
           const int row = b * dec.page + jt * BN;
 #pragma unroll
@@ -341,7 +289,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
         if (lane < n) {
           const int key = jt * BN + lane * box;
           int row = static_cast<int>(dec.cache_rows);
-          if (key < sq.len) {
+          if (key < len) {
             if (blk >= 0 && static_cast<long long>(blk + 1) * dec.page <= dec.cache_rows)
               row = blk * dec.page + key % dec.page;
             else
@@ -357,20 +305,12 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      if constexpr (!DEC) {
-        const int row_q = sq.start + m_blk * BM;
-        mbar_arrive_expect_tx(bars.q(), C::QK_TILE);
+      // q_len tokens x g heads: one (64, g, q_len) box per column block.
+      mbar_arrive_expect_tx(bars.q(), dec.n_rows * 128 * C::CHUNKS);
 #pragma unroll
-        for (int c = 0; c < C::QK_CHUNKS; ++c)
-          tma_load_2d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), h * D + c * 64, row_q);
-      } else {
-        // q_len tokens x g heads: one (64, g, q_len) box per column block.
-        mbar_arrive_expect_tx(bars.q(), dec.n_rows * 128 * C::CHUNKS);
-#pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), c * 64, hk * dec.g,
-                      b * dec.q_len);
-      }
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_load_3d(sbase + C::OFF_Q + c * CHUNK_BYTES, &tm_q, bars.q(), c * 64, hk * dec.g,
+                    b * dec.q_len);
     }
     // K and V run through separate rings and are loaded independently, K
     // first whenever both have a free slot: K_j is consumed early (QK_j runs
@@ -389,9 +329,9 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
           __all_sync(FULL, mbar_try_wait(bars.k_empty(jk % C::STAGES),
                                          ((jk / C::STAGES) & 1) ^ 1))) {
         const int st = jk % C::STAGES;
-        if (lane == 0) mbar_arrive_expect_tx(bars.k_full(st), C::QK_TILE);
+        if (lane == 0) mbar_arrive_expect_tx(bars.k_full(st), C::TILE);
         __syncwarp();
-        load_kv(sbase + C::OFF_K + st * C::QK_TILE, &tm_k, bars.k_full(st), j0 + jk, kpb, true);
+        load_kv(sbase + C::OFF_K + st * C::TILE, &tm_k, bars.k_full(st), j0 + jk, kpb);
         ++jk;
         progress = true;
       }
@@ -401,7 +341,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
         const int st = jv % C::STAGES;
         if (lane == 0) mbar_arrive_expect_tx(bars.v_full(st), C::TILE);
         __syncwarp();
-        load_kv(sbase + C::OFF_V + st * C::TILE, &tm_v, bars.v_full(st), j0 + jv, vpb, false);
+        load_kv(sbase + C::OFF_V + st * C::TILE, &tm_v, bars.v_full(st), j0 + jv, vpb);
         ++jv;
         progress = true;
       }
@@ -428,7 +368,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       const int t = n_kv - 1;
       const int st = t % C::STAGES;
       if (warp_wait(bars.v_full(st), (t / C::STAGES) & 1, p.err, abort, W_VTAIL)) {
-        const int first = sq.len - (j0 + t) * BN;   // rows [first, 128) are past the end
+        const int first = len - (j0 + t) * BN;   // rows [first, 128) are past the end
         uint8_t* tile = smem + C::OFF_V + st * C::TILE;
         for (int i = lane; i < (BN - first) * 8 * C::CHUNKS; i += 32) {
           const int c = i / ((BN - first) * 8);
@@ -467,10 +407,8 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     const bool do_pv = !C::SPLIT_MMA || warp == WARP_PV;
     const uint32_t leader = elect_one();
     constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
-    constexpr uint32_t IDESC_QK8 = idesc_e4m3(BM, BN);
     constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
     const uint64_t k_desc = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
-    const uint64_t q_desc = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);   // E4M3 path only
     const uint64_t v_desc = sdesc_sw128(sbase + C::OFF_V, CHUNK_BYTES, 1024);
     // Q reaches TMEM through the softmax threads.
     bool ok = warp_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM);
@@ -488,19 +426,11 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_s = tmem + TM_S0 + (jq & 1) * BN;
-        if constexpr (F8) {
-          // M=128, N=128, K=D in steps of 32 codes (32 bytes of a row).
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)
-            mma_ss_e4m3_if(leader, d_s, sdesc_add(q_desc, kk * 32),
-                           sdesc_add(k_desc, st * C::QK_TILE + kk * 32), IDESC_QK8, kk > 0);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-            mma_ts_if(leader, d_s, tmem + TM_Q + kk * 8,
-                      sdesc_add(k_desc, st * C::QK_TILE + off), IDESC_QK, kk > 0);
-          }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
+          mma_ts_if(leader, d_s, tmem + TM_Q + kk * 8, sdesc_add(k_desc, st * C::TILE + off),
+                    IDESC_QK, kk > 0);
         }
         tc_commit_if(leader, bars.s_full(jq & 1));
         tc_commit_if(leader, bars.k_empty(st));
@@ -526,31 +456,16 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     const int g = warp >> 2;            // softmax group: key tiles g, g+2, ...
     const int quarter = warp & 3;       // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    // Last visible key of this row (-1: none) and whether the row is output.
-    int lim;
-    bool row_ok;
-    size_t out_row;   // row index of O / LSE in units of heads
-    if constexpr (!DEC) {
-      const int qpos = m_blk * BM + row;
-      lim = p.causal ? min(qpos, sq.len - 1) : sq.len - 1;
-      row_ok = qpos < sq.len;
-      out_row = static_cast<size_t>(sq.start + qpos) * p.H + h;
-    } else {
-      // Row r is query token r / g (position len - q_len + r / g of the
-      // sequence) of query head hk * g + r % g.
-      row_ok = row < dec.n_rows;
-      const int pos = sq.len - dec.q_len + row / dec.g;
-      lim = !row_ok ? -1 : (p.causal ? min(pos, sq.len - 1) : sq.len - 1);
-      out_row = static_cast<size_t>(b * dec.q_len + row / dec.g) * p.H + hk * dec.g + row % dec.g;
-    }
+    // Row r is query token r / g (position len - q_len + r / g of the
+    // sequence) of query head hk * g + r % g. lim: last visible key of this
+    // row (-1: none); out_row: row index of O / LSE in units of heads.
+    const bool row_ok = row < dec.n_rows;
+    const int pos = len - dec.q_len + row / dec.g;
+    const int lim = !row_ok ? -1 : (p.causal ? min(pos, len - 1) : len - 1);
+    const size_t out_row =
+        static_cast<size_t>(b * dec.q_len + row / dec.g) * p.H + hk * dec.g + row % dec.g;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    float c2 = p.scale_log2;
-    // E4M3 scores are in units of Delta_Q Delta_K of their two blocks.
-    const float* kscale_row = nullptr;
-    if constexpr (F8) {
-      c2 *= __ldg(f8.q_scale + (static_cast<size_t>(b) * p.H + h) * f8.n_blocks + m_blk);
-      kscale_row = f8.k_scale + (static_cast<size_t>(b) * p.H_kv + hk) * f8.n_blocks;
-    }
+    const float c2 = p.scale_log2;   // log2 units per raw score
     float* mref_s = reinterpret_cast<float*>(smem + C::OFF_MREF);
     float* fin_s = reinterpret_cast<float*>(smem + C::OFF_FIN);
     float m_g = -INFINITY;  // reference of this group's last tile (log2 units)
@@ -560,17 +475,15 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       // Copy this row of Q from the swizzled shared tile into TMEM as packed
       // bf16 (even element in the low half): the A operand of S = Q K^T.
       ok = warp_wait(bars.q(), 0, p.err, abort, W_Q);
-      if (ok && F8) {
-        mbar_arrive(bars.q_tmem());   // the E4M3 score MMA reads Q from shared memory
-      } else if (ok) {
+      if (ok) {
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c) {
           const uint8_t* rowp = smem + C::OFF_Q + c * CHUNK_BYTES + row * 128;
           uint32_t w[32];
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) {
-            // Decode rows past the q_len x g block were never loaded: zeros.
-            const uint4 v = (DEC && !row_ok)
+            // Rows past the q_len x g block were never loaded: zeros.
+            const uint4 v = !row_ok
                                 ? make_uint4(0, 0, 0, 0)
                                 : *reinterpret_cast<const uint4*>(rowp + ((k16 ^ (row & 7)) << 4));
             w[4 * k16 + 0] = v.x;
@@ -589,14 +502,13 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       // group 1 writes none before group 0 has finished copying Q out of it.
       ok = warp_wait(bars.q_tmem(), 0, p.err, abort, W_QTMEM);
     }
-    // Decode warps whose 32 rows are all padding (q_len x g < 128) keep the
+    // Warps whose 32 rows are all padding (q_len x g < 128) keep the
     // barrier protocol - the same waits and arrivals, in the same order, so
     // no barrier phase ever mixes two tiles - but load, exponentiate and
     // store nothing: their rows are never written out.
-    const bool idle = DEC && __all_sync(FULL, !row_ok);
+    const bool idle = __all_sync(FULL, !row_ok);
     for (int j = g; j < n_kv && ok; j += 2) {
       const uint32_t s_col = TM_S0 + g * BN;
-      const float c2t = F8 ? c2 * __ldg(kscale_row + j) : c2;   // log2 units per raw score
       if (!warp_wait(bars.s_full(g), (j >> 1) & 1, p.err, abort, W_SFULL)) {
         ok = false;
         break;
@@ -657,7 +569,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       // The reference only moves when the row max exceeds it by more than
       // RESCALE_LOG2 (log2 units): P = 2^(s c - m_ref) then stays below
       // 2^RESCALE_LOG2, and O / l is the same for any consistent reference.
-      const float m_cand = mx * c2t;
+      const float m_cand = mx * c2;
       const bool grow = m_cand > m_prev + RESCALE_LOG2;   // always true on tile 0
       const float m_new = grow ? m_cand : m_prev;
       mref_s[g * BM + row] = m_new;
@@ -669,8 +581,8 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2t, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2t, -m_use));
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][i]), c2, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use));
           sum4[(i >> 1) & 3] += p0 + p1;
           pk[c >> 1][(c & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
         }
@@ -730,8 +642,8 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       if (m_o != -INFINITY) l += (m_o == m_fin) ? l_o : l_o * ex2_approx(m_o - m_fin);
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       const float lse = (l > 0.f) ? (m_fin + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      // Split partials (decode with several splits) stay fp32 for the merge.
-      const bool part = DEC && dec.n_split > 1;
+      // Split partials (several splits) stay fp32 for the merge.
+      const bool part = dec.n_split > 1;
       const size_t prow = static_cast<size_t>(split) * p.total * p.H + out_row;
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
@@ -763,9 +675,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
         }
       }
       if (row_ok && g == 0) {
-        if constexpr (!DEC)
-          p.lse[lse_index(p, b, h, sq.start, m_blk * BM + row)] = lse;
-        else if (part)
+        if (part)
           dec.lse_part[prow] = lse;
         else
           p.lse[out_row] = lse;
@@ -821,51 +731,8 @@ __global__ void __launch_bounds__(256)
 }
 
 template <int D>
-cudaError_t launch_d(const AttnParams& p, cudaStream_t stream) {
-  using C = FwdCfg<D, false>;
-  const int num_m = (p.max_seqlen + BM - 1) / BM;
-  const long long tiles = static_cast<long long>(num_m) * p.H * p.B;
-  if (tiles == 0 || p.total == 0) return cudaSuccess;
-  if (tiles > INT_MAX) return cudaErrorInvalidConfiguration;
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap_bf16_2d(&tq, p.q, p.total, static_cast<unsigned long long>(p.H) * D, 64, BM) ||
-      !make_tmap_bf16_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN) ||
-      !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, false, false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  const int group = l2_group(4ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_bf16_kernel<D, false, false><<<static_cast<unsigned>(tiles), C::THREADS, C::SMEM, stream>>>(
-      tq, tk, tv, p, num_m, group, DecodeArgs{}, Fp8Args{});
-  return cudaGetLastError();
-}
-
-// E4M3 forward: p.q / p.k hold the codes, ``f`` their per-block steps.
-cudaError_t launch_fp8_d128(const AttnParams& p, const Fp8Args& f, cudaStream_t stream) {
-  constexpr int D = 128;
-  using C = FwdCfg<D, true>;
-  const int num_m = (p.max_seqlen + BM - 1) / BM;
-  const long long tiles = static_cast<long long>(num_m) * p.H * p.B;
-  if (tiles == 0 || p.total == 0) return cudaSuccess;
-  if (tiles > INT_MAX) return cudaErrorInvalidConfiguration;
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap_u8_2d(&tq, p.q, p.total, static_cast<unsigned long long>(p.H) * D, 128, BM) ||
-      !make_tmap_u8_2d(&tk, p.k, p.total, static_cast<unsigned long long>(p.H_kv) * D, 128, BN) ||
-      !make_tmap_bf16_2d(&tv, p.v, p.total, static_cast<unsigned long long>(p.H_kv) * D, 64, BN))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, false, true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  const int group = l2_group(3ll * p.max_seqlen * D, p.H / p.H_kv, p.H * p.B);
-  fwd_bf16_kernel<D, false, true><<<static_cast<unsigned>(tiles), C::THREADS, C::SMEM, stream>>>(
-      tq, tk, tv, p, num_m, group, DecodeArgs{}, f);
-  return cudaGetLastError();
-}
-
-template <int D>
 cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream) {
-  using C = FwdCfg<D, false>;
+  using C = Cfg<D>;
   const long long ctas = static_cast<long long>(p.B) * p.H_kv * d.n_split;
   if (ctas == 0) return cudaSuccess;
   if (ctas > INT_MAX) return cudaErrorInvalidConfiguration;
@@ -878,11 +745,11 @@ cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream
       !make_tmap_bf16_2d(&tv, p.v, d.cache_rows, static_cast<unsigned long long>(p.H_kv) * D, 64,
                          box_rows))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<D, true, false>,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  fwd_bf16_kernel<D, true, false><<<static_cast<unsigned>(ctas), C::THREADS, C::SMEM, stream>>>(
-      tq, tk, tv, p, 0, 0, d, Fp8Args{});
+  decode_split_kernel<D><<<static_cast<unsigned>(ctas), C::THREADS, C::SMEM, stream>>>(
+      tq, tk, tv, p, d);
   e = cudaGetLastError();
   if (e != cudaSuccess || d.n_split == 1) return e;
   const long long rows = p.total * p.H;
@@ -892,21 +759,6 @@ cudaError_t launch_decode_d(const AttnParams& p, const DecodeArgs& d, cudaStream
 }
 
 }  // namespace
-
-cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream) {
-  // D = 128: two query tiles per CTA (fwd_pair.cu). D = 64 is bound by the
-  // exponentials (half the tensor work per score), where the larger CTA only
-  // lengthens the last wave: measured 0.146 ms here against 0.153 ms for the
-  // two-tile kernel on B4 H16 N2048.
-  if (p.D == 64) return launch_d<64>(p, stream);
-  if (p.D == 128) return launch_fwd_pair(p, stream);
-  return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_fwd_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream) {
-  if (p.D == 128) return launch_fp8_d128(p, f, stream);
-  return cudaErrorInvalidValue;
-}
 
 cudaError_t launch_decode_bf16(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream) {
   if (p.D == 64) return launch_decode_d<64>(p, d, stream);

@@ -7,7 +7,7 @@
 // online-softmax recurrence of aiqz.cc "Flash Attention V2/V3 optimization",
 // section "V2 algorithm optimisation", and the partials of a segment are
 // merged with the same update. Two things differ from the one-CTA-per-split
-// kernel in fwd_bf16.cu.
+// kernel in decode_split.cu.
 //
 // The cut. The units (sequence b, kv head, 128-key tile) are numbered in
 // that order and cut into one contiguous range of equal size per SM, so

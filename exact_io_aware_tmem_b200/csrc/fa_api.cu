@@ -10,7 +10,6 @@
 #include "../../include/fa.h"
 #include "decode_t.h"
 #include "fwd_d64.h"
-#include "fwd_fp8.h"
 #include "params.h"
 
 namespace fa {
@@ -236,7 +235,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const cudaError_t e = (dtype == FA_F32) ? fa::launch_fwd_f32(p, s)
                         : (D == 64)       ? fa::launch_fwd_d64(p, s)
-                                          : fa::launch_fwd_bf16(p, s);
+                                          : fa::launch_fwd_pair(p, s);
   return fa::cuda_status(e);
 }
 

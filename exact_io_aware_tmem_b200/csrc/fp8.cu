@@ -4,7 +4,7 @@
 // precision": the first pass scans each block in high precision for its
 // largest |x|, sets the block's step Delta = max|x| / 448 (448 is E4M3's
 // largest finite value) and stores round(x / Delta) as E4M3; the second pass
-// (fwd_bf16.cu, F8 instantiation) multiplies the codes on the tensor cores
+// (fwd_pair.cu, F8 instantiation) multiplies the codes on the tensor cores
 // with an fp32 accumulator.
 //
 // A block is the 128 consecutive tokens of one head of one sequence - one

@@ -1,7 +1,7 @@
 // Attention forward at D = 64, bf16 in / fp32 accumulate: one 128-row query
 // tile per CTA, one softmax group, two CTAs per SM.
 //
-// What it computes is the forward of fwd_bf16.cu: for every query row the
+// What it computes is the forward of fwd_pair.cu: for every query row the
 // online-softmax recurrence of aiqz.cc "Flash Attention V2/V3 optimization",
 // section "V2 algorithm optimisation" (steps 1-5), over key tiles j,
 //     m_new = max(m, rowmax(S_j)), l = l e^(m - m_new) + rowsum(e^(S_j - m_new)),
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 }  // namespace d64
 }  // namespace
 
-// The D = 64 forward (launch_fwd_bf16 uses it).
+// The D = 64 forward (fa_fwd uses it).
 cudaError_t launch_fwd_d64(const AttnParams& p, cudaStream_t stream) {
   using namespace d64;
   if (p.D != D) return cudaErrorInvalidValue;

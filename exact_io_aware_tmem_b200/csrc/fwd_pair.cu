@@ -1,5 +1,5 @@
 // Attention forward, two 128-row query tiles per CTA, bf16 in / fp32
-// accumulate, on the sm_100a tensor cores (D = 64 and 128).
+// accumulate, on the sm_100a tensor cores (D = 128).
 //
 // What it computes: for every query row, the online-softmax recurrence of
 // aiqz.cc "Flash Attention V2/V3 optimization", section "V2 algorithm
@@ -40,7 +40,6 @@
 #include <limits.h>
 #include <math.h>
 
-#include "fwd_fp8.h"
 #include "params.h"
 
 namespace fa {
@@ -62,7 +61,7 @@ constexpr int VS_MAX = 4;
 
 template <int D, bool F8>
 struct Cfg {
-  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(D == 128, "head dim (D = 64 has its own kernel, fwd_d64.cu)");
   static_assert(!F8 || D == 128, "E4M3 rows of 128 bytes");
   static constexpr uint32_t TILE = BM * D * 2;       // bf16 tile, 32 KB at D = 128
   static constexpr uint32_t QK_TILE = F8 ? BM * D : TILE;   // Q or K tile
@@ -533,7 +532,6 @@ cudaError_t launch_fwd_pair_fp8(const AttnParams& p, const Fp8Args& f, cudaStrea
 }
 
 cudaError_t launch_fwd_pair(const AttnParams& p, cudaStream_t stream) {
-  if (p.D == 64) return launch_pair_d<64>(p, stream);
   if (p.D == 128) return launch_pair_d<128>(p, stream);
   return cudaErrorInvalidValue;
 }

@@ -154,8 +154,7 @@ struct Fp8Args {
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_f32(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_f32(const AttnParams& p, cudaStream_t stream);
-cudaError_t launch_fwd_bf16(const AttnParams& p, cudaStream_t stream);
-// The D = 128 forward with two query tiles per CTA (launch_fwd_bf16 uses it).
+// The D = 128 forward, two query tiles per CTA (fwd_pair.cu).
 cudaError_t launch_fwd_pair(const AttnParams& p, cudaStream_t stream);
 // mask: bit 0 preprocess (D_i, and zeroes dq_accum when it is set), bit 1
 // dK/dV kernel, bit 2 dQ kernel (the split backward).
@@ -165,12 +164,14 @@ cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned m
 cudaError_t launch_bwd_fused(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_dq_convert(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
-// E4M3 forward (D = 128) on codes from launch_fp8_quantize.
-cudaError_t launch_fwd_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream);
+// E4M3 forward (D = 128) on the same kernel: p.q / p.k hold the codes from
+// launch_fp8_quantize, ``f`` their per-block steps.
+cudaError_t launch_fwd_pair_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream);
 // Pass 1: bf16 x [B*N, Hx, D] -> E4M3 codes x8 and per-block steps [B, Hx, nb].
 cudaError_t launch_fp8_quantize(const void* x, void* x8, float* scale, int B, int N, int Hx,
                                 int D, cudaStream_t stream);
-// Decode partials (and the combine kernel when d.n_split > 1).
+// Split-KV decode partials (decode_split.cu), and the combine kernel when
+// d.n_split > 1.
 cudaError_t launch_decode_bf16(const AttnParams& p, const DecodeArgs& d, cudaStream_t stream);
 
 // Host: the argument checks fa_bwd applies to the sizes (status as fa_bwd
