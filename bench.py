@@ -123,8 +123,8 @@ def source_sha(*names) -> str:
 
 
 KERNEL_SOURCES = {"fwd_pair_kernel": ("fwd_pair.cu", "common.cuh", "params.h"),
-                  "fwd_d64_kernel": ("fwd_d64.cu", "fwd_d64.h", "common.cuh", "params.h"),
-                  "bwd_fused_kernel": ("bwd_fused.cu", "common.cuh", "params.h"),
+                  "fwd_d64_kernel": ("fwd_d64.cu", "fwd_d64.h", "ex2_fma.cuh", "common.cuh", "params.h"),
+                  "bwd_fused_kernel": ("bwd_fused.cu", "ex2_fma.cuh", "common.cuh", "params.h"),
                   "bwd_dkdv_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "bwd_dq_kernel": ("bwd_bf16.cu", "common.cuh", "params.h"),
                   "decode": ("decode_split.cu", "common.cuh", "params.h"),

@@ -54,6 +54,7 @@ SIGNATURES = {
     "fa_check_device_error": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_uint)]),
     "fa_set_wait_budget": (None, [c_ll]),
     "fa_selftest_wait_timeout": (c_int, [c_ll, c_void_p]),
+    "fa_selftest_exp2": (c_int, [c_void_p, c_void_p, c_ll, c_void_p]),
     "fa_decode_num_splits": (c_int, [c_int, c_int, c_int, c_int]),
     "fa_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int, c_int]),
     "fa_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,

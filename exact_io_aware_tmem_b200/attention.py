@@ -232,6 +232,17 @@ def selftest_wait_timeout(cycles: int, device: Optional[torch.device] = None) ->
                "fa_selftest_wait_timeout")
 
 
+def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
+    """2^x by the kernels' FMA-pipe exponential (fa_selftest_exp2), for a
+    contiguous fp32 CUDA tensor."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("selftest_exp2 takes a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    _abi.check(_lib().fa_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(x.device)),
+               "fa_selftest_exp2")
+    return y
+
+
 def set_wait_budget(cycles: int) -> None:
     _lib().fa_set_wait_budget(int(cycles))
 

@@ -10,6 +10,7 @@
 #include "../../include/fa.h"
 #include "decode_t.h"
 #include "fwd_d64.h"
+#include "ex2_fma.cuh"
 #include "params.h"
 
 namespace fa {
@@ -204,6 +205,25 @@ __global__ void wait_selftest_kernel(DevErr e) {
 
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(err);
+  return cudaGetLastError();
+}
+
+namespace {
+
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                     long long n) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += stride)
+    y[i] = ex2_fma(x[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_exp2_selftest(const float* x, float* y, long long n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const long long blocks = std::min<long long>((n + 255) / 256, 148 * 8);
+  exp2_selftest_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, y, n);
   return cudaGetLastError();
 }
 
@@ -504,6 +524,11 @@ fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream) {
   return fa::launch_wait_selftest(e, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? FA_OK
              : FA_ERR_CUDA;
+}
+
+fa_status fa_selftest_exp2(const float* x, float* y, long long n, fa_stream_t stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return FA_ERR_INVALID_ARG;
+  return fa::cuda_status(fa::launch_exp2_selftest(x, y, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 const char* fa_last_cuda_error_string(void) { return cudaGetErrorString(fa::g_last_cuda); }

@@ -164,6 +164,7 @@ cudaError_t launch_bwd_bf16(const AttnParams& p, cudaStream_t stream, unsigned m
 cudaError_t launch_bwd_fused(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_dq_convert(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DevErr err, cudaStream_t stream);
+cudaError_t launch_exp2_selftest(const float* x, float* y, long long n, cudaStream_t stream);
 // E4M3 forward (D = 128) on the same kernel: p.q / p.k hold the codes from
 // launch_fp8_quantize, ``f`` their per-block steps.
 cudaError_t launch_fwd_pair_fp8(const AttnParams& p, const Fp8Args& f, cudaStream_t stream);

@@ -266,6 +266,17 @@ void fa_set_wait_budget(long long cycles);
 fa_status fa_selftest_wait_timeout(long long cycles, fa_stream_t stream);
 
 /*
+ * fa_selftest_exp2 - y[i] = 2^x[i] for n device floats, by the FMA-pipe
+ * exponential that the D = 64 forward and the fused backward use for a
+ * share of their softmax exponentials (range reduction x = n + f, |f| <= 1/2,
+ * and a degree-3 minimax polynomial for 2^f: relative error at most 7.5e-5
+ * for -125 <= x <= 127; x <= -126, -inf included, gives about 2^-126).
+ * Enqueued on ``stream``. FA_ERR_INVALID_ARG for n < 0 or null pointers
+ * with n > 0.
+ */
+fa_status fa_selftest_exp2(const float* x, float* y, long long n, fa_stream_t stream);
+
+/*
  * Debug build. The library built with -DFA_DEBUG (libfa_b200_debug.so, same
  * entry points) checks indices in its kernels against the buffers they
  * address, recording a failed check in the device error word
