@@ -78,6 +78,32 @@ struct Bars {
   __device__ uint32_t pv_done() const { return b + 8u * (4 + 2 * KSTAGES + 2 * VSTAGES); }
 };
 
+// Debug builds: event kinds of the traced CTA's stamps (one per key tile j;
+// T_W_EPI once, at index 0), and every CTA's SM and global timer (ns) at its
+// start and end (kinds 29-31, at index blockIdx.x), whichever CTA is traced.
+enum : int {
+  T_W_SFULL = 0, T_W_LD = 1, T_W_EXP = 2, T_W_ARR = 3, T_M_S = 4, T_M_PV = 5, T_W_EPI = 6,
+  T_CTA_SM = 29, T_CTA_START = 30, T_CTA_END = 31
+};
+
+__device__ __forceinline__ void cta_span(const AttnParams& p, int kind) {
+#ifdef FA_DEBUG
+  if (p.trace != nullptr && blockIdx.x < 1024) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    p.trace[kind * 1024 + blockIdx.x] = t;
+    if (kind == T_CTA_START) {
+      unsigned sm;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+      p.trace[T_CTA_SM * 1024 + blockIdx.x] = sm + 1ull;
+    }
+  }
+#else
+  (void)p;
+  (void)kind;
+#endif
+}
+
 // Codes recorded in the device error word when a wait gives up.
 enum : unsigned {
   W_Q = 0x80100, W_KEMPTY = 0x80200, W_VEMPTY = 0x80300, W_KFULL = 0x80400, W_VFULL = 0x80500,
@@ -121,6 +147,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int b = ts.unit / p.H;
   const SeqInfo sq = seq_info(p, b);
   if (!seq_ok(p, sq) || m_blk * BM >= sq.len) return;   // whole CTA, before any shared state
+  if (threadIdx.x == 0) cta_span(p, T_CTA_START);
   const int hk = h / (p.H / p.H_kv);
   const int n_kv_all = (sq.len + BN - 1) / BN;
   const int n_kv = p.causal ? min(n_kv_all, m_blk + 1) : n_kv_all;
@@ -250,6 +277,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                     sdesc_add(k_desc, st * TILE + kk * 32), IDESC_QK, kk > 0);
         tc_commit_if(leader, bars.s_full());
         tc_commit_if(leader, bars.k_empty(st));
+        if (lane == 0) FA_STAMP(p, T_M_S, is);
         ++is;
         progress = true;
       }
@@ -264,6 +292,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                     (ip > 0 || kk > 0) ? 1u : 0u);
         tc_commit_if(leader, bars.v_empty(st));
         tc_commit_if(leader, bars.pv_done());
+        if (lane == 0) FA_STAMP(p, T_M_PV, ip);
         ++ip;
         progress = true;
       }
@@ -291,11 +320,13 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int lim = p.causal ? min(qpos, sq.len - 1) : sq.len - 1;   // last visible key
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float c2 = p.scale_log2;
+    const bool stamp = threadIdx.x == 0;   // debug stamps: lane 0 of warp 0
     float m_ref = -INFINITY;   // reference max (log2 units)
     float l = 0.f;             // row sum in that reference
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
       if (!(ok = warp_wait(bars.s_full(), j & 1, p.err, abort, W_SFULL))) break;
+      if (stamp) FA_STAMP(p, T_W_SFULL, j);
       tc_fence_after();
       uint32_t r[4][32];
 #pragma unroll
@@ -303,6 +334,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+      if (stamp) FA_STAMP(p, T_W_LD, j);
       // The scores are in registers: the tensor core may overwrite S.
       tc_fence_before();
       mbar_arrive(bars.s_free());
@@ -348,6 +380,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           pk[c >> 1][(c & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
         }
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      if (stamp) FA_STAMP(p, T_W_EXP, j);
       const float alpha = (grow && m_prev != -INFINITY) ? ex2_approx(m_prev - m_use) : 1.f;
       l = grow ? l * alpha + sum : l + sum;
       // P_{j-1} V_{j-1} has read P and added into O.
@@ -372,6 +405,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bars.p_ready());
+      if (stamp) FA_STAMP(p, T_W_ARR, j);
     }
     // ----------------------------------------------------------- epilogue ---
     const int last = n_kv - 1;
@@ -405,6 +439,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         }
       }
       if (row_ok) p.lse[lse_index(p, b, h, sq.start, qpos)] = lse;
+      if (stamp) FA_STAMP(p, T_W_EPI, 0);
     }
   }
 
@@ -414,6 +449,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  if (threadIdx.x == 0) cta_span(p, T_CTA_END);
 }
 
 }  // namespace d64

@@ -11,6 +11,11 @@ what.
   python -m exact_io_aware_tmem_b200.trace --kernel bwd --workload NAME [--cta 0]
   python -m exact_io_aware_tmem_b200.trace --kernel fwd --workload NAME
   python -m exact_io_aware_tmem_b200.trace --kernel dec --workload DECODE_NAME
+  python -m exact_io_aware_tmem_b200.trace --kernel d64 --workload bf16_fwd_b4_h16_n2048_d64
+
+The balanced decode and the D = 64 forward also record every CTA's SM and
+global-timer span (the first 1024 CTAs): how long CTAs take, and how much of
+each SM's time they cover.
 
 The traced CTA is blockIdx.x (0: the first launched, with the longest causal
 work).
@@ -38,6 +43,9 @@ FWD_KINDS = {
 }
 DEC_KINDS = {
     "P_K": 0, "P_V": 1, "M_S": 2, "M_PV": 3, "W_SFULL": 4, "W_ARR": 5, "W_EPI": 6,
+}
+D64_KINDS = {
+    "W_SFULL": 0, "W_LD": 1, "W_EXP": 2, "W_ARR": 3, "M_S": 4, "M_PV": 5, "W_EPI": 6,
 }
 # (label, from event, step offset of from, to event, step offset of to): the
 # median of stamp[to][t + dto] - stamp[from][t + dfrom] over the steps t.
@@ -95,7 +103,6 @@ FWD_SPANS = [
 
 # Per-CTA records of the balanced decode (index = CTA): SM + 1, and the
 # global timer (ns) at the CTA's start and end.
-DEC_CTA_SM, DEC_CTA_START, DEC_CTA_END = 29, 30, 31
 
 DEC_SPANS = [
     ("producer: K_j issued -> S_j issued (K landed, S buffer free)", "P_K", 0, "M_S", 0),
@@ -109,6 +116,54 @@ DEC_SPANS = [
     ("producer: K_{j+3} issued after S_j issued (slot refill)", "M_S", 0, "P_K", 3),
     ("producer: V_{j+3} issued after P_j V_j issued (slot refill)", "M_PV", 0, "P_V", 3),
 ]
+
+
+D64_SPANS = [
+    ("softmax: S_j seen -> scores in registers", "W_SFULL", 0, "W_LD", 0),
+    ("softmax: scores in registers -> exponentials done", "W_LD", 0, "W_EXP", 0),
+    ("softmax: exponentials done -> P_j published", "W_EXP", 0, "W_ARR", 0),
+    ("softmax: P_j published -> S_{j+1} seen", "W_ARR", 0, "W_SFULL", 1),
+    ("softmax: tile period (S_j seen -> S_{j+1} seen)", "W_SFULL", 0, "W_SFULL", 1),
+    ("MMA warp: scores of S_j read -> S_{j+1} issued", "W_LD", 0, "M_S", 1),
+    ("tensor: S_j issued -> softmax sees S_j", "M_S", 0, "W_SFULL", 0),
+    ("MMA warp: P_j published -> P_j V_j issued", "W_ARR", 0, "M_PV", 0),
+]
+CTA_SM, CTA_START, CTA_END = 29, 30, 31
+
+
+def cta_report(stamps) -> list:
+    """Lines on the CTAs' global-timer spans: count, durations, and per SM the
+    CTA time over the wall time (mean CTAs resident) and the share of the
+    wall time with at least one CTA resident."""
+    st = stamps[CTA_START].astype(np.int64)
+    en = stamps[CTA_END].astype(np.int64)
+    sm = stamps[CTA_SM].astype(np.int64) - 1
+    ok = (st != 0) & (en != 0) & (sm >= 0)
+    if not ok.any():
+        return []
+    st, en, sm = st[ok], en[ok], sm[ok]
+    t0, t1 = st.min(), en.max()
+    wall = max(int(t1 - t0), 1)
+    dur = (en - st) / 1e3
+    lines = [f"  CTAs: {int(ok.sum())}, all done {wall / 1e3:.1f} us after the first started; "
+             f"start spread {(st.max() - t0) / 1e3:.1f} us; duration min {dur.min():.1f} "
+             f"median {np.median(dur):.1f} max {dur.max():.1f} us"]
+    resident, covered = [], []
+    for s in np.unique(sm):
+        a, b = st[sm == s], en[sm == s]
+        resident.append(float((b - a).sum()) / wall)
+        ev = sorted([(int(x), 1) for x in a] + [(int(y), -1) for y in b])
+        live, last, cov = 0, int(t0), 0
+        for t, d in ev:
+            if live > 0:
+                cov += t - last
+            live += d
+            last = t
+        covered.append(cov / wall)
+    lines.append(f"  SMs: {len(resident)}; mean CTAs resident {statistics.fmean(resident):.2f} "
+                 f"(min {min(resident):.2f}); time with a CTA resident "
+                 f"{100 * statistics.fmean(covered):.1f} % (min {100 * min(covered):.1f} %)")
+    return lines
 
 
 def spans(stamps, kinds: dict, table, n_steps: int, skip: int = 2) -> list:
@@ -180,6 +235,8 @@ def run(kernel: str, workload: str, cta: int = 0):
 
     if kernel == "dec":
         return run_decode(workload, cta)
+    if kernel == "d64" and WORKLOADS[workload].D != 64:
+        raise ValueError("--kernel d64 takes a D = 64 workload")
 
     w = WORKLOADS[workload]
     inp = make_inputs(w)
@@ -197,7 +254,7 @@ def run(kernel: str, workload: str, cta: int = 0):
     buf = torch.zeros(_abi.DEBUG_TRACE_BYTES // 8, dtype=torch.int64, device=dev)
     with fa.debug_build() as lib:
         assert lib.fa_debug_build() == 1
-        if kernel == "fwd":
+        if kernel in ("fwd", "d64"):
             _abi.check(lib.fa_debug_set_trace(buf.data_ptr(), buf.numel() * 8, cta), "trace")
             o, lse = fa.fwd(q, k, v, **kw)
             _abi.check(lib.fa_debug_set_trace(None, 0, 0), "trace")
@@ -217,15 +274,15 @@ def run(kernel: str, workload: str, cta: int = 0):
     stamps = buf.view(32, 1024).cpu().numpy()
     # Steps of the traced CTA: query steps (backward) or key tiles (forward;
     # the second query tile of a causal pair has one more than the first).
-    firsts = ["S_SFULL"] if kernel == "bwd" else ["W0_SFULL", "W1_SFULL"]
-    kinds = BWD_KINDS if kernel == "bwd" else FWD_KINDS
+    firsts = {"bwd": ["S_SFULL"], "fwd": ["W0_SFULL", "W1_SFULL"], "d64": ["W_SFULL"]}[kernel]
+    kinds = {"bwd": BWD_KINDS, "fwd": FWD_KINDS, "d64": D64_KINDS}[kernel]
     n = max(int((stamps[kinds[f]] != 0).sum()) for f in firsts)
     return stamps, n
 
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("--kernel", choices=["fwd", "bwd", "dec"], required=True)
+    ap.add_argument("--kernel", choices=["fwd", "bwd", "dec", "d64"], required=True)
     ap.add_argument("--workload", default="bf16_causal_b2_h16_n8192_d128")
     ap.add_argument("--cta", type=int, default=0)
     args = ap.parse_args(argv)
@@ -233,20 +290,14 @@ def main(argv=None) -> int:
     build(debug=True)
     stamps, n = run(args.kernel, args.workload, args.cta)
     kinds, table = {"bwd": (BWD_KINDS, BWD_SPANS), "fwd": (FWD_KINDS, FWD_SPANS),
-                    "dec": (DEC_KINDS, DEC_SPANS)}[args.kernel]
+                    "dec": (DEC_KINDS, DEC_SPANS), "d64": (D64_KINDS, D64_SPANS)}[args.kernel]
     print(f"{args.kernel} {args.workload} CTA {args.cta}: {n} steps stamped; cycles over "
           f"the steady-state steps")
-    if args.kernel == "dec":
-        st, en = stamps[DEC_CTA_START].astype(np.int64), stamps[DEC_CTA_END].astype(np.int64)
-        ok = (st != 0) & (en != 0)
-        if ok.any():
-            t0 = st[ok].min()
-            dur = (en[ok] - st[ok]) / 1e3
-            print(f"  CTAs: {int(ok.sum())}, all done {(en[ok].max() - t0) / 1e3:.1f} us after the "
-                  f"first started; start spread {(st[ok].max() - t0) / 1e3:.1f} us; duration "
-                  f"min {dur.min():.1f} median {np.median(dur):.1f} max {dur.max():.1f} us")
+    if args.kernel in ("dec", "d64"):
+        for line in cta_report(stamps):
+            print(line)
         stamps = stamps.copy()
-        stamps[DEC_CTA_SM:DEC_CTA_END + 1] = 0
+        stamps[CTA_SM:CTA_END + 1] = 0
     nz = stamps[stamps != 0]
     if nz.size:
         span = int(nz.max()) - int(nz.min())

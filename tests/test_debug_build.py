@@ -106,7 +106,48 @@ def test_debug_build_decode_stamps(debug_lib):
     assert (np.diff(s) > 0).all()
     # every CTA's SM and span
     sm, st, en = (stamps[k][:groups * w.H_kv].astype(np.int64)
-                  for k in (trace.DEC_CTA_SM, trace.DEC_CTA_START, trace.DEC_CTA_END))
+                  for k in (trace.CTA_SM, trace.CTA_START, trace.CTA_END))
     assert (sm >= 1).all() and (sm <= 148).all() and (en > st).all() and (st > 0).all()
     for label, med, mean, p90, cnt in trace.spans(stamps, trace.DEC_KINDS, trace.DEC_SPANS, n):
         assert med is not None and cnt > 0, label
+    assert trace.cta_report(stamps)
+
+
+@pytest.mark.gpu
+def test_debug_build_d64_stamps(debug_lib):
+    """The D = 64 forward on B4 H16 N2048: the traced CTA stamps its 16 key
+    tiles in order, and all 1024 CTAs record their SM and span, at most two
+    resident per SM at a time."""
+    name = "bf16_fwd_b4_h16_n2048_d64"
+    stamps, n = trace.run("d64", name, cta=3)
+    assert n == 16
+    s = stamps[trace.D64_KINDS["W_ARR"]][:n].astype(np.int64)
+    assert (np.diff(s) > 0).all()
+    sm, st, en = (stamps[k].astype(np.int64) for k in (trace.CTA_SM, trace.CTA_START,
+                                                         trace.CTA_END))
+    assert (sm >= 1).all() and (sm <= 148).all() and (en > st).all() and (st > 0).all()
+    for s_id in np.unique(sm):
+        ev = sorted([(int(a), 1) for a in st[sm == s_id]] + [(int(b), -1) for b in en[sm == s_id]],
+                    key=lambda e: (e[0], e[1]))
+        live = np.cumsum([d for _, d in ev])
+        assert live.max() <= 2, s_id
+    for label, med, mean, p90, cnt in trace.spans(stamps, trace.D64_KINDS, trace.D64_SPANS, n):
+        assert med is not None and cnt > 0, label
+    assert trace.cta_report(stamps)
+
+
+def test_cta_report_host_arithmetic():
+    """cta_report on hand-made spans: two SMs over a 100 us wall, SM 0 with
+    two CTAs back to back (covered all the time, one resident on average),
+    SM 1 with one CTA for the first half."""
+    stamps = np.zeros((32, 1024), dtype=np.int64)
+    rows = [(0, 0, 50_000), (0, 50_000, 100_000), (1, 0, 50_000)]
+    for i, (s, a, b) in enumerate(rows):
+        stamps[trace.CTA_SM][i] = s + 1
+        stamps[trace.CTA_START][i] = 1_000 + a
+        stamps[trace.CTA_END][i] = 1_000 + b
+    lines = trace.cta_report(stamps)
+    assert "CTAs: 3, all done 100.0 us" in lines[0]
+    assert "median 50.0" in lines[0]
+    assert "SMs: 2; mean CTAs resident 0.75 (min 0.50)" in lines[1]
+    assert "time with a CTA resident 75.0 % (min 50.0 %)" in lines[1]
