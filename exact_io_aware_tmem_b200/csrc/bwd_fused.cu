@@ -104,8 +104,8 @@ struct Cfg {
   static constexpr uint32_t OFF_DO = OFF_Q + QS * TILE;
   static constexpr uint32_t OFF_DS = OFF_DO + GS * TILE;       // dS^T: 128 keys x 128 queries bf16
   static constexpr uint32_t OFF_STG = OFF_DS + 2 * SPAN;       // dQ staging: 8 KB per dQ warp
-  static constexpr uint32_t OFF_LSE = OFF_STG + 8 * 4096;      // float [QS][BT]: LSE * log2(e)
-  static constexpr uint32_t OFF_DLT = OFF_LSE + QS * BT * 4;   // float [QS][BT]: D_i
+  static constexpr uint32_t OFF_LSE = OFF_STG + 8 * 4096;      // float [QS][BT]: -LSE * log2(e)
+  static constexpr uint32_t OFF_DLT = OFF_LSE + QS * BT * 4;   // float [QS][BT]: -D_i
   static constexpr uint32_t OFF_BAR = OFF_DLT + QS * BT * 4;
   // kv_full, q_full[QS], q_empty[QS], do_full[GS], do_empty[GS], s_full,
   // dp_full, p_ready, ds_ready, dq_full, dq_free, dkv_done
@@ -342,8 +342,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
 #pragma unroll
       for (int k = 0; k < BT / 32; ++k) {
-        s_lse[st * BT + lane + 32 * k] = pl[k] * LOG2E;
-        s_dlt[st * BT + lane + 32 * k] = pd[k];
+        // Negated, so the dS warps add them in packed fp32 pairs.
+        s_lse[st * BT + lane + 32 * k] = -(pl[k] * LOG2E);
+        s_dlt[st * BT + lane + 32 * k] = -pd[k];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.q_full(st));
@@ -583,8 +584,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           // An eighth of the exponentials (2 of every 16 queries) on the
           // FMA pipe: warps w and w + 4 share each sub-partition's
           // special-function unit (-1.5 to -4 % on the backward).
-          const float x0 = fmaf(__uint_as_float(sr[q]), c2, -la);
-          const float x1 = fmaf(__uint_as_float(sr[q + 1]), c2, -lb);
+          // Pairs of scores on the packed fp32 FMA path (la, lb hold -LSE log2 e).
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[q]), __uint_as_float(sr[q + 1])),
+                                      make_float2(c2, c2), make_float2(la, lb));
+          const float x0 = x.x, x1 = x.y;
           const bool fma_pipe = (q % 16) == 0;
           float p0 = fma_pipe ? ex2_fma(x0) : ex2_approx(x0);
           float p1 = fma_pipe ? ex2_fma(x1) : ex2_approx(x1);
@@ -626,8 +629,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t w = pk[16 * c + (q >> 1)];
           const float p0 = __uint_as_float(w << 16);
           const float p1 = __uint_as_float(w & 0xffff0000u);
-          dsk[16 * c + (q >> 1)] = pack_bf16x2(p0 * (__uint_as_float(dr[q]) - da),
-                                               p1 * (__uint_as_float(dr[q + 1]) - db));
+          // dS = P (dP - D) on packed pairs (da, db hold -D).
+          const float2 v = __fmul2_rn(
+              make_float2(p0, p1),
+              __fadd2_rn(make_float2(__uint_as_float(dr[q]), __uint_as_float(dr[q + 1])),
+                         make_float2(da, db)));
+          dsk[16 * c + (q >> 1)] = pack_bf16x2(v.x, v.y);
         }
       }
       // dS^T into the shared dS^T tile: the A operand of dQ (read MN-major)
