@@ -361,25 +361,27 @@ __global__ void __launch_bounds__(THREADS, 2)
       const float m_prev = m_ref;
       if (grow) m_ref = m_cand;
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      // Arguments and row sums on packed fp32 pairs (0.1188 against 0.1208 ms).
+      float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 c2p = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
       uint32_t pk[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
+          const float2 x =
+              __ffma2_rn(make_float2(__uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1])), c2p, nm);
           // A quarter of the exponentials (4 of every 16 keys) on the FMA
           // pipe: the two CTAs' softmax warps share each sub-partition's
           // special-function unit (0.1208 against 0.1249 ms on B4 H16 N2048;
           // an eighth 0.1229, three eighths 0.1311).
-          const float x0 = fmaf(__uint_as_float(r[c][i]), c2, -m_use);
-          const float x1 = fmaf(__uint_as_float(r[c][i + 1]), c2, -m_use);
           const bool fma_pipe = (i % 16) < 4;
-          const float p0 = fma_pipe ? ex2_fma(x0) : ex2_approx(x0);
-          const float p1 = fma_pipe ? ex2_fma(x1) : ex2_approx(x1);
-          sum4[(i >> 1) & 3] += p0 + p1;
+          const float p0 = fma_pipe ? ex2_fma(x.x) : ex2_approx(x.x);
+          const float p1 = fma_pipe ? ex2_fma(x.y) : ex2_approx(x.y);
+          sum2[(i >> 1) & 1] = __fadd2_rn(sum2[(i >> 1) & 1], make_float2(p0, p1));
           pk[c >> 1][(c & 1) * 16 + i / 2] = pack_bf16x2(p0, p1);
         }
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      const float sum = (sum2[0].x + sum2[1].x) + (sum2[0].y + sum2[1].y);
       if (stamp) FA_STAMP(p, T_W_EXP, j);
       const float alpha = (grow && m_prev != -INFINITY) ? ex2_approx(m_prev - m_use) : 1.f;
       l = grow ? l * alpha + sum : l + sum;
