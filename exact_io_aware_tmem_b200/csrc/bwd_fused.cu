@@ -36,11 +36,11 @@
 // At D = 64 dQ_t has columns of its own.
 //
 // Roles (512 threads, four warpgroups):
-//   warps 0-7   dS warps (warpgroups 0, 1; 128 registers). Thread = key row
+//   warps 0-7   dS warps (warpgroups 0, 1; 136 registers). Thread = key row
 //               (TMEM lane) for S^T / dP^T, warps w and w+4 taking query
 //               columns [64 hf, 64 hf + 64). Per step: exponentials of S^T_t
 //               -> P^T_t into TMEM, then dS^T_t into the shared dS tile.
-//   warps 8-11  dQ warps (warpgroup 2; 176 registers, enough to hold a whole
+//   warps 8-11  dQ warps (warpgroup 2; 160 registers, enough to hold a whole
 //               row block of dQ_t). Thread = query row of dQ_t (TMEM lane):
 //               the read-out in one go, dq_free, then the staging and the
 //               reductions, off the dS warps' path. With the read-out this
@@ -79,11 +79,14 @@ constexpr int WARP_TMA = 12;   // warpgroup 3: producer, MMA warp, two idle warp
 constexpr int WARP_MMA = 13;
 // Registers per thread (setmaxnreg): the block launches at 128 (16 warps,
 // four per SM sub-partition, 16K registers each). Warpgroup 3 gives back 48
-// of them per thread and the dQ warps take them, enough to hold a whole dQ_t
-// row block: 2 x 128 + 176 + 80 = 4 x 128 on every sub-partition and for the
-// block.
-constexpr uint32_t REG_DQ = 176;
+// of them per thread; the dQ warps take 32 (160: a whole dQ_t row block in
+// registers) and each dS warpgroup 8 (136: nothing spills, where at 128 the
+// dS warps' packed arithmetic did; -2.5 % on causal N8192).
+// 2 x 136 + 160 + 80 = 4 x 128 on every sub-partition and for the block.
+constexpr uint32_t REG_DS = 136;
+constexpr uint32_t REG_DQ = 160;
 constexpr uint32_t REG_CTRL = 80;
+static_assert(2 * REG_DS + REG_DQ + REG_CTRL == 4 * 128, "register split of the block");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr unsigned FULL = 0xffffffffu;
 constexpr uint32_t SPAN = BT * 128;   // 128 rows x 128 bytes: one 128-byte swizzle column block
@@ -536,6 +539,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) bulk_wait_all();
     __syncwarp();
   } else {
+    regs_inc<REG_DS>();
     // ------------------------------------------------------------ dS warps ---
     // Key-side work: thread = key row r (TMEM lane); warps w and w+4 take the
     // query columns [64 hf, 64 hf + 64) of the step.
